@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of one decode layer's hot path on B200: act-quant -> FC_QKV +
+attention scaling -> split-KV attention with cluster DSMEM merge -> act-quant ->
+FC13 + SwiGLU, PDL-chained, all in libdl.so.
+
+Default workload: the batch-1 decode layer (1 token, FC_QKV 5120->7168,
+FC13 5120->2x8192, attention 40/8 heads d=128 over 4096 cached keys).  Inputs
+are synthetic and seeded.  Every timed step runs on a different copy of the
+layer (weights and KV cache), and one rotation over the copies moves more than
+three times the 126 MB L2, so each step streams its weights and KV from HBM.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on the
+same workload instead (the deliberately slow reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs per decode layer; achieved HBM TB/s vs B200 peak (FP8 GEMM, split-KV attn)"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="layer_b1")
+    p.add_argument("--cluster", type=int, default=0, help="attention cluster size (0 = workload default)")
+    p.add_argument("--replicas", type=int, default=0, help="layer copies to rotate through (0 = auto)")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline sample length")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def env_int(name, default):
+    v = os.environ.get(name)
+    return int(v) if v is not None else default
+
+
+def workload_config(wl, cluster):
+    return {"workload": f"{wl.name}: M={wl.M} K={wl.K} FC_QKV N={wl.n_qkv} FC13 N2={wl.N2} "
+                        f"attn B={wl.B} T={wl.T} Hq={wl.Hq} Hkv={wl.Hkv} d={wl.d} L={wl.L} cluster={cluster}",
+            "tokens": wl.M, "hidden": wl.K, "kv_len": wl.L, "heads_q": wl.Hq, "heads_kv": wl.Hkv,
+            "head_dim": wl.d, "cluster": cluster,
+            "l2": "inputs larger than L2: each step uses another layer copy; one rotation > 3x L2"}
+
+
+# ---------------------------------------------------------------- oracle arm --
+
+def oracle_layer_inputs(wl):
+    from latency_decode_b200 import datagen as dg
+    return dg.dense_layer_inputs(wl)
+
+
+def oracle_layer(wl, inp):
+    """One layer through the CPU oracle (same steps as the GPU path)."""
+    import numpy as np
+    import oracle
+    from latency_decode_b200 import datagen as dg
+    qkv = oracle.fc_qkv_scale(inp["x1"], inp["w_qkv"], inp["s_qkv"], wl.Hq, wl.Hkv, wl.d, inp["q_scale"])
+    qb = dg.bf16_bits(qkv.astype(np.float32))
+    oracle.decode_attn(qb.ravel(), wl.n_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, inp["k_cache"], inp["v_cache"],
+                       inp["seq_lens"], 1.0)
+    oracle.fc13_swiglu(inp["x2"], inp["w13"], inp["s13"])
+
+
+def time_oracle(wl, inp, seconds, min_reps=1, max_reps=10**6):
+    reps, t0 = 0, time.perf_counter()
+    while reps < min_reps or (time.perf_counter() - t0 < seconds and reps < max_reps):
+        oracle_layer(wl, inp)
+        reps += 1
+    dt = time.perf_counter() - t0
+    return dt / reps * 1e6, reps, dt
+
+
+def run_reference(args):
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    from latency_decode_b200 import datagen as dg
+    wl = dg.WORKLOADS[args.workload]
+    cluster = args.cluster or wl.cluster
+    inp = oracle_layer_inputs(wl)
+    for _ in range(args.warmup):
+        oracle_layer(wl, inp)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_layer(wl, inp)
+        times.append(time.perf_counter() - t0)
+    us = sum(times) / len(times) * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, cluster),
+        "cpu_baseline": {"value": us, "unit": "us", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} full {wl.name} layers (QKV GEMM, attention, FC13) "
+                                   "through the single-threaded FP64 C++ oracle"},
+        "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- clocks --------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------- GPU arm --------
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def make_layers(wl, R, seed_base, device, cluster):
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200.layer import DecodeLayer
+    import numpy as np
+    layers, kvs, xs = [], [], []
+    g = dg.rng(wl.seed)
+    sl = dg.seq_lens_for(wl, g)
+    seq_lens = torch.from_numpy(sl).to(device)
+    for r in range(R):
+        gen = torch.Generator(device=device).manual_seed(seed_base + r)
+        wq, sq = dg.e4m3_weight_torch(gen, wl.n_qkv, wl.K, device)
+        w13, s13 = dg.e4m3_weight_torch(gen, wl.N2, wl.K, device)
+        layer = DecodeLayer(wq, sq, w13, s13, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, q_scale=1.0 / math.sqrt(wl.d),
+                            M=wl.M, B=wl.B, T=wl.T, cluster=cluster, device=device)
+        del wq, w13
+        kc = torch.randn((wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device).to(torch.bfloat16)
+        vc = torch.randn((wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device).to(torch.bfloat16)
+        x1 = torch.randn((wl.M, wl.K), generator=gen, device=device).to(torch.bfloat16)
+        x2 = torch.randn((wl.M, wl.K), generator=gen, device=device).to(torch.bfloat16)
+        layers.append(layer)
+        kvs.append((kc.view(torch.int16), vc.view(torch.int16)))
+        xs.append((x1.view(torch.int16), x2.view(torch.int16)))
+    torch.cuda.synchronize()
+    return layers, kvs, xs, seq_lens, sl
+
+
+def timed(fn, steps, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        fn(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)  # ms
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from latency_decode_b200 import build as dl_build
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200 import dl
+
+    rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU for --impl ours")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    dl_build.build()
+    dl.lib()
+
+    wl = dg.WORKLOADS[args.workload]
+    cluster = args.cluster or wl.cluster
+    per_layer = wl.n_qkv * wl.K + wl.N2 * wl.K + 2 * wl.B * wl.Hkv * wl.Lcap * wl.d * 2
+    R = args.replicas or max(2, math.ceil(3 * L2_BYTES / per_layer))
+    layers, kvs, xs, seq_lens, sl = make_layers(wl, R, 1000 * (rank + 1), device, cluster)
+    stream = torch.cuda.current_stream()
+    h = stream.cuda_stream
+
+    def step(i, flags=dl.DL_FLAG_PDL):
+        r = i % R
+        layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens, stream=h, flags=flags)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    for lay in layers:
+        lay.read_status(h)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    # ---- timed region: K whole-layer steps ----
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    ms = timed(step, args.steps, stream)
+    barrier()
+    clk = clocks.stop()
+    for lay in layers:
+        lay.read_status(h)
+    us_layer = ms * 1e3 / args.steps
+    if world > 1:
+        t = torch.tensor([us_layer], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        us_layer = float(t.item())
+
+    # ---- the same steps without PDL (context) ----
+    us_layer_nopdl = timed(lambda i: step(i, 0), args.steps, stream) * 1e3 / args.steps
+
+    # ---- per-call loops, for the roofline of each kernel family ----
+    K = wl.K
+    def call_qkv(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_fc_qkv_scale(xs[r][0], wl.M, K, L_.wp_qkv, L_.s_qkv, wl.Hq, wl.Hkv, wl.d, L_.q_scale, L_.qkv,
+                                    L_.ws_qkv, stream=h))
+
+    def call_attn(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_decode_attn(L_.qkv, L_.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, kvs[r][0], kvs[r][1],
+                                   wl.Lcap, seq_lens, 1.0, cluster, L_.attn_out, L_.ws_attn, stream=h))
+
+    def call_fc13(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_fc13_swiglu(xs[r][1], wl.M, K, L_.wp_13, L_.s_13, wl.N2, L_.ffn_out, L_.ws_13, stream=h))
+
+    kv_bytes = int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
+    fam = {
+        "fc13_swiglu": (call_fc13, wl.N2 * wl.K, 2),
+        "fc_qkv_scale": (call_qkv, wl.n_qkv * wl.K, 2),
+        "decode_attn": (call_attn, kv_bytes, 1),
+    }
+    peak, peak_kind = peak_hbm()
+    kernels = {}
+    for name, (fn, nbytes, launches) in fam.items():
+        for i in range(3):
+            fn(i)
+        us = timed(fn, args.steps, stream) * 1e3 / args.steps
+        gbs = nbytes / (us * 1e-6) / 1e9
+        kernels[name] = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak,
+                         "launches_per_call": launches}
+    for lay in layers:
+        lay.read_status(h)
+
+    # ---- end to end through the public API with host buffers ----
+    r0 = 0
+    hx1 = torch.empty_like(xs[0][0], device="cpu").pin_memory()
+    hx2 = torch.empty_like(xs[0][1], device="cpu").pin_memory()
+    hx1.copy_(xs[0][0].cpu())
+    hx2.copy_(xs[0][1].cpu())
+    ha = torch.empty_like(layers[0].attn_out, device="cpu").pin_memory()
+    hf = torch.empty_like(layers[0].ffn_out, device="cpu").pin_memory()
+    dx1 = [torch.empty_like(xs[r][0]) for r in range(R)]
+    dx2 = [torch.empty_like(xs[r][1]) for r in range(R)]
+
+    def e2e_step(i):
+        r = i % R
+        dx1[r].copy_(hx1, non_blocking=True)
+        dx2[r].copy_(hx2, non_blocking=True)
+        layers[r].step(dx1[r], dx2[r], kvs[r][0], kvs[r][1], seq_lens, stream=h)
+        ha.copy_(layers[r].attn_out, non_blocking=True)
+        hf.copy_(layers[r].ffn_out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    us_e2e = timed(e2e_step, args.steps, stream) * 1e3 / args.steps
+    if world > 1:
+        t = torch.tensor([us_e2e], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        us_e2e = float(t.item())
+    h2d = hx1.numel() * 2 + hx2.numel() * 2
+    d2h = ha.numel() * 2 + hf.numel() * 2
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        inp = oracle_layer_inputs(wl)
+        us_cpu, reps, secs = time_oracle(wl, inp, args.cpu_seconds, min_reps=1)
+        cpu = {"value": us_cpu, "unit": "us", "cores": 1, "kind": "oracle",
+               "sample": f"{reps} full {wl.name} layers ({secs:.1f} s) through the single-threaded FP64 C++ "
+                         "oracle on the host"}
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    dom = kernels["fc13_swiglu"]
+    line = {
+        "metric": METRIC, "value": us_layer, "unit": "us", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us_layer / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8e4m3xfp8e4m3->f32 GEMM, bf16 attention (f32 softmax)",
+        "data": "synthetic", "config": workload_config(wl, cluster),
+        "roofline": {"bound": "hbm", "kernel": "fc13_swiglu (act-quant + tcgen05 FP8 GEMM + SwiGLU)",
+                     "achieved": dom["achieved_gbs"], "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": dom["achieved_gbs"] / peak, "traffic": None},
+        "kernels": kernels,
+        "layer_us_no_pdl": us_layer_nopdl,
+        "layer_alg_bytes": wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes,
+        "layer_achieved_gbs": (wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes) / (us_layer * 1e-6) / 1e9,
+        "e2e": {"value": us_e2e, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "cpu_baseline": cpu,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk,
+        "replicas": R,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,198 @@
+/*
+ * dl.h -- C ABI of libdl.so, the B200 (sm_100a) low-latency FP8 decode kernels.
+ *
+ * The library implements the decode hot path described by the NVIDIA technical
+ * blog "Blackwell breaks the 1,000 TPS/user barrier with Meta's Llama 4
+ * Maverick" (cited below as [NV], Korean edition) and its Chinese rewrite by
+ * Xinzhiyuan (cited as [XZY]):
+ *   - an FP8 (e4m3, per-tensor scale) weight-streaming GEMM at tiny M with two
+ *     fused epilogues, FC13+SwiGLU and FC_QKV+attention scaling, plus a grouped
+ *     per-expert (MoE) variant;
+ *   - grouped-query decode attention split along the KV sequence, whose per-block
+ *     partial softmax states are merged across a thread-block cluster through
+ *     distributed shared memory;
+ *   - consecutive kernels chained with Programmatic Dependent Launch.
+ *
+ * Conventions that hold for every entry point
+ * -------------------------------------------
+ * - Every data pointer is a DEVICE pointer unless stated otherwise; the caller
+ *   allocates and owns every buffer.  The library never allocates, frees or
+ *   synchronises in these calls (dl_read_status is the one call that
+ *   synchronises the stream).
+ * - bf16 tensors are passed as their raw 16-bit patterns (uint16_t); e4m3
+ *   tensors as raw bytes (uint8_t, OCP FP8 E4M3 "e4m3fn" encoding).
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * - Errors the host can see (null pointers, shapes, alignment, workspace size)
+ *   are returned BEFORE anything is launched.  A failed launch returns
+ *   DL_ERR_CUDA.  Errors only the device can see (a bounded wait that ran out,
+ *   a sequence length or expert id out of range) are OR-ed into the status
+ *   word of the workspace and reported by dl_read_status; the outputs of that
+ *   call are then undefined.
+ * - Outputs are written in full on success.
+ * - With DL_FLAG_PDL each kernel is launched with programmatic stream
+ *   serialisation.  Every kernel of this library waits for its predecessor
+ *   before it triggers its own dependents, and reads only "static" inputs
+ *   (packed weights, weight scales, KV cache, sequence lengths, expert ids)
+ *   before that wait.  Hence: with DL_FLAG_PDL, those static inputs must not be
+ *   outputs of the kernel that immediately precedes the call in the stream
+ *   when that kernel is itself one of this library's kernels.
+ * - Workspace: `ws` is device memory of at least dl_workspace_bytes(...) bytes,
+ *   256-byte aligned, zero-filled by the caller once before first use.  Layout:
+ *     [0, 4)        uint32 status word (bits: 1 timeout, 2 bad sequence length,
+ *                   4 bad expert id); cleared by dl_read_status
+ *     [8, 12)       float  s_x, the activation scale of the last GEMM call
+ *     [256, 256+M*K) uint8 x_q, the e4m3 activations [M][K] of the last GEMM call
+ *   Two calls that may run concurrently (or overlap under PDL) must not share
+ *   a workspace.
+ */
+#ifndef LATENCY_DECODE_DL_H
+#define LATENCY_DECODE_DL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dl_status {
+  DL_OK = 0,
+  DL_ERR_INVALID_ARG = 1,   /* null pointer, shape or range error (host-side) */
+  DL_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement */
+  DL_ERR_ALIGNMENT = 3,     /* a pointer or stride is not aligned as required */
+  DL_ERR_WORKSPACE = 4,     /* ws is null, misaligned or smaller than required */
+  DL_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+  DL_ERR_TIMEOUT = 6,       /* a bounded device wait ran out (from dl_read_status) */
+  DL_ERR_DEVICE_ARG = 7     /* the device found a bad seq_len / expert id (from dl_read_status) */
+} dl_status;
+
+/* flags (bitwise OR) */
+#define DL_FLAG_PDL 1u            /* launch with Programmatic Dependent Launch */
+#define DL_FLAG_DEBUG_TIMEOUT 2u  /* test hook: shortens every bounded wait to ~2 ms and
+                                     withholds the last pipeline load, so the consumer's
+                                     wait runs out and DL_ERR_TIMEOUT is reported */
+#define DL_FLAG_SPLIT_SHIFT 8     /* bits [8,13): if non-zero, force the GEMM split-K
+                                     cluster size (1..8) instead of the built-in choice */
+
+/* weight pack kinds */
+#define DL_PACK_PLAIN 0   /* FC_QKV and other plain projections */
+#define DL_PACK_SWIGLU 1  /* FC13: gate rows [0,F) and up rows [F,2F) paired per tile */
+
+/* ---------------------------------------------------------------------------
+ * Offline weight swizzle.  [XZY] "CUDA 内核优化与融合", item "GEMM 权重重排";
+ * [NV] "CUDA kernel optimisation and fusion": the GEMM weights are rearranged
+ * offline into a swizzled layout so that the result read back from Tensor
+ * Memory after the tensor-core MMA lands in a convenient order.
+ *
+ * Input  w_nk: canonical e4m3 weight, row-major [N][K] (nn.Linear layout).
+ * Output w_packed: N*K bytes.  Let KB = K/128.  The packed tensor is a
+ * sequence of 16384-byte blocks; each block is the shared-memory image of 128
+ * weight rows x 128 K-bytes in the tcgen05 K-major 128-byte-swizzle layout:
+ * byte c of row r sits at (r/8)*1024 + (r%8)*128 + ((c/16) ^ (r%8))*16 + c%16.
+ *   DL_PACK_PLAIN  (N % 128 == 0): block (t*KB + kb) holds rows 128t..128t+127,
+ *                  K-bytes 128kb..128kb+127.
+ *   DL_PACK_SWIGLU (N % 256 == 0, F = N/2): block 2*(t*KB + kb) holds gate rows
+ *                  128t..128t+127 and block 2*(t*KB + kb)+1 the up rows
+ *                  F+128t..F+128t+127, for the same K-bytes.  The gate and up
+ *                  accumulators of one output column then land in the same
+ *                  Tensor Memory lane, so SwiGLU needs no data exchange.
+ * Requirements: K % 128 == 0, pointers 16-byte aligned, w_nk and w_packed must
+ * not overlap.  The pack is an exact byte permutation.
+ * ------------------------------------------------------------------------- */
+dl_status dl_pack_fp8_weight(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
+                             void* stream);
+
+/* Bytes of workspace a GEMM call with M rows of K activations needs
+ * (256 + M*K rounded up to 256).  dl_workspace_bytes(0, 0) = 256 is what
+ * dl_decode_attn needs (the status word only). */
+size_t dl_workspace_bytes(int M, int K);
+
+/* ---------------------------------------------------------------------------
+ * FC13 + SwiGLU.  [XZY] "运算融合" and [NV] fusion list: SwiGLU is fused into
+ * the GEMM before it; the activation Quantize is fused ahead of the GEMM.
+ *   x       bf16 [M][K], row-major, 16-byte aligned
+ *   w_packed e4m3, DL_PACK_SWIGLU layout of the [N2][K] weight, 16-byte aligned
+ *   w_scale device float[1], the per-tensor weight scale s_w
+ *   out     bf16 [M][N2/2], row-major, 16-byte aligned
+ * Computes s_x and x_q = e4m3(x / s_x) (one dynamic per-tensor scale,
+ * s_x = max|x| / 448), y = s_x * s_w * x_q . W^T accumulated in fp32 on the
+ * tensor cores, and out[m][j] = silu(y[m][j]) * y[m][F+j] rounded to bf16.
+ * Supported: 1 <= M <= 64, K % 128 == 0, N2 % 256 == 0.
+ * ------------------------------------------------------------------------- */
+dl_status dl_fc13_swiglu(const uint16_t* x, int M, int K, const uint8_t* w_packed,
+                         const float* w_scale, int N2, uint16_t* out, void* ws,
+                         size_t ws_bytes, void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * FC_QKV + attention scaling.  [XZY] "运算融合"; [NV] fusion list.
+ *   w_packed e4m3, DL_PACK_PLAIN layout of the [(Hq+2*Hkv)*d][K] weight
+ *   qkv     bf16 [M][(Hq+2*Hkv)*d], row-major: Q heads, then K heads, then V heads
+ * y as above; the Q columns [0, Hq*d) are multiplied by q_scale (normally
+ * 1/sqrt(d)), the K and V columns are not.  Supported: 1 <= M <= 64,
+ * K % 128 == 0, (Hq+2*Hkv)*d % 128 == 0.
+ * ------------------------------------------------------------------------- */
+dl_status dl_fc_qkv_scale(const uint16_t* x, int M, int K, const uint8_t* w_packed,
+                          const float* w_scale, int Hq, int Hkv, int d, float q_scale,
+                          uint16_t* qkv, void* ws, size_t ws_bytes, void* stream,
+                          unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * Grouped MoE expert FC13 + SwiGLU, top-1.  [XZY] FP8 for GEMM, MoE and
+ * attention; [NV] "CUDA kernel optimisation and fusion" (MoE kernels).
+ *   x          bf16 [T][K]
+ *   expert_ids device int32[T], each in [0, E)
+ *   w_packed   E consecutive DL_PACK_SWIGLU blocks of N2*K bytes (expert e at
+ *              byte offset e*N2*K)
+ *   w_scales   device float[E]
+ *   out        bf16 [T][N2/2], rows in token order
+ * One activation scale over all T tokens.  Token t uses expert expert_ids[t].
+ * Only the experts that some token selects are read from memory.  Routing is
+ * computed on the device from expert_ids (no host synchronisation).
+ * Supported: 1 <= T <= 64, 1 <= E <= 1024, K % 128 == 0, N2 % 256 == 0.
+ * ------------------------------------------------------------------------- */
+dl_status dl_moe_fc13_swiglu_grouped(const uint16_t* x, int T, int K, const int32_t* expert_ids,
+                                     int E, const uint8_t* w_packed, const float* w_scales,
+                                     int N2, uint16_t* out, void* ws, size_t ws_bytes,
+                                     void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * Split-KV grouped-query decode attention with a cluster DSMEM merge.
+ * [XZY] "CUDA 内核优化与融合", item "Attention内核并行优化"; [NV] "CUDA kernel
+ * optimisation and fusion": the work is split along the sequence dimension of
+ * K and V over several thread blocks, and the blocks of one thread-block
+ * cluster reduce their partial results through distributed shared memory
+ * instead of global memory.
+ *   q         bf16, q[b][t][h][i] at q[(b*T + t)*q_token_stride + h*d + i]
+ *             (q may point into the qkv output of dl_fc_qkv_scale, with
+ *             q_token_stride = (Hq+2*Hkv)*d and softmax_scale = 1, since those
+ *             Q columns are already scaled)
+ *   k_cache, v_cache  bf16 [B][Hkv][Lcap][d], contiguous, 16-byte aligned
+ *   seq_lens  device int32[B]; sequence b has L = seq_lens[b] keys, the last T
+ *             of which are the new tokens: query t sees keys 0 .. L-T+t
+ *             (bottom-right causal).  T <= L <= Lcap is required (checked on
+ *             the device: DL_ERR_DEVICE_ARG from dl_read_status, output zero).
+ *   out       bf16 [B][T][Hq][d], contiguous
+ * o = softmax(softmax_scale * q K^T) V per (b, t, head); q head h reads kv
+ * head h / (Hq/Hkv).  Each (b, kv head) is handled by one cluster of
+ * cluster_size CTAs (1, 2, 4, 8 or 16); CTA r streams the r-th contiguous
+ * chunk of ceil(L/cluster_size) keys (rounded up to 16).
+ * Supported: d in {64, 128}, Hq % Hkv == 0, (Hq/Hkv)*T <= 32, q_token_stride
+ * a multiple of 8 and >= Hq*d.
+ * ------------------------------------------------------------------------- */
+dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int T, int Hq,
+                         int Hkv, int d, const uint16_t* k_cache, const uint16_t* v_cache,
+                         int Lcap, const int32_t* seq_lens, float softmax_scale,
+                         int cluster_size, uint16_t* out, void* ws, size_t ws_bytes,
+                         void* stream, unsigned flags);
+
+/* Synchronises `stream`, reads the status word of `ws`, clears it, and returns
+ * DL_OK, DL_ERR_TIMEOUT or DL_ERR_DEVICE_ARG (timeout takes precedence). */
+dl_status dl_read_status(void* ws, void* stream);
+
+/* A static, human-readable name of a status code. */
+const char* dl_status_string(dl_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LATENCY_DECODE_DL_H */

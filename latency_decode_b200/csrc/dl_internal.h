@@ -1,0 +1,89 @@
+// dl_internal.h -- host-side declarations shared by the .cu files of libdl.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dl.h"
+
+namespace dl {
+
+// Fills the launch attributes for an optional cluster shape and PDL.
+struct Launch {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[2];
+  Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster_x, bool pdl) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    int n = 0;
+    if (cluster_x > 0) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = cluster_x;
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+    if (pdl) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+  }
+};
+
+int sm_count();  // SMs of the current device (cached per device)
+
+// Workspace layout (see dl.h).
+constexpr size_t kWsHeader = 256;
+inline uint32_t* ws_status(void* ws) { return static_cast<uint32_t*>(ws); }
+inline float* ws_sx(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 8); }
+inline uint8_t* ws_xq(void* ws) { return static_cast<uint8_t*>(ws) + kWsHeader; }
+
+// ---- kernels' host launchers (return a CUDA error code) ----
+cudaError_t launch_act_quant(const uint16_t* x, int M, int K, uint8_t* xq, float* s_x,
+                             cudaStream_t s, bool pdl);
+cudaError_t launch_pack(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
+                        cudaStream_t s);
+
+struct GemmLaunch {
+  const uint8_t* w;
+  long long w_expert_bytes;
+  const float* w_scale;
+  const uint8_t* xq;
+  const float* s_x;
+  uint32_t* status;
+  uint16_t* out;
+  const int32_t* expert_ids;  // null for dense
+  int M, K, N, ldo, E;        // N = output rows streamed per expert (N2 for SwiGLU)
+  int q_cols;
+  float q_scale;
+  bool swiglu;
+  int slots;                  // grid z (1 for dense)
+  int split;                  // forced split-K cluster size (0 = choose)
+  bool debug;
+  bool pdl;
+};
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s);
+
+struct AttnLaunch {
+  const uint16_t* q;
+  long long q_stride;
+  int B, T, Hq, Hkv, d, Lcap;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* seq_lens;
+  float scale;
+  int cluster;
+  uint16_t* out;
+  uint32_t* status;
+  bool debug;
+  bool pdl;
+};
+cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t s);
+
+}  // namespace dl

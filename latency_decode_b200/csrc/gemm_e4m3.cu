@@ -1,0 +1,403 @@
+// gemm_e4m3.cu -- A2/A5/A6: FP8 (e4m3, per-tensor scale) weight-streaming
+// GEMM at tiny M on the 5th-generation tensor cores, with the FC13+SwiGLU and
+// FC_QKV+attention-scaling epilogues and the grouped per-expert (MoE) variant.
+//
+// Sources: [XZY] "CUDA 内核优化与融合" (items "空间分区与高效内存加载" -- warp
+// specialisation so weight loads use the HBM bandwidth, "GEMM 权重重排" -- the
+// offline weight swizzle, "运算融合" -- SwiGLU fused into the GEMM); [NV]
+// "CUDA kernel optimisation and fusion" (low-latency GEMM kernels, FC13 +
+// SwiGLU and FC_QKV + attn_scaling fusions, FP8 MoE).
+//
+// Design (B200-native; the pages give no code):
+//  * swap-AB: the weight tile (128 output rows x 128 K-bytes) is the M=128
+//    operand A of tcgen05.mma.kind::f8f6f4, the few tokens are the N operand
+//    (N = tokens rounded up to 8), the fp32 accumulator lives in Tensor Memory
+//    with one output row per TMEM lane.
+//  * weights are pre-swizzled offline (pack.cu), so one 16 KB cp.async.bulk per
+//    pipeline stage lands a ready tcgen05 operand in shared memory.
+//  * warp roles: warp 0 streams weights through a ring of 16 KB stages (it does
+//    not wait for the preceding kernel: weights are static, so under PDL the
+//    ring fills while the predecessor still runs), warp 1 issues the MMAs,
+//    warps 2-3 stage the activations into the swizzled B operand; all four
+//    warps then read the accumulators back with tcgen05.ld.
+//  * split-K over a cluster of S CTAs: each CTA reduces 1/S of K, the S partial
+//    accumulators are summed through distributed shared memory (each CTA owns
+//    128/S output rows), and the nonlinear epilogue runs on the full sums.
+//  * SwiGLU: the gate rows and the up rows of the same output columns are two
+//    MMAs into two TMEM column ranges of the same lanes, so one thread holds
+//    both g and u of its output and applies silu(g)*u directly.
+//  * MoE: grid z is an expert slot; every CTA derives the slot's expert and its
+//    tokens from expert_ids on the device (no host sync), and CTAs of unused
+//    slots exit at once, so only touched experts are read from HBM.
+#include <cuda_bf16.h>
+
+#include "dl_device.cuh"
+#include "dl_internal.h"
+
+namespace dl {
+
+constexpr int kGemmThreads = 128;
+constexpr int kSubBytes = 16384;  // one packed block: 128 rows x 128 K-bytes
+constexpr int kMaxTok = 64;
+constexpr int kMaxExperts = 1024;
+
+struct GemmArgs {
+  const uint8_t* w;           // packed weights (expert 0 block for MoE)
+  long long w_expert_bytes;   // bytes per expert block (0 for dense)
+  const float* w_scale;       // [1] or [E]
+  const uint8_t* xq;          // e4m3 activations [M][K]
+  const float* s_x;           // activation scale
+  uint32_t* status;
+  uint16_t* out;              // bf16 [tokens][ldo]
+  const int32_t* expert_ids;  // MoE routing (null for dense)
+  int M, K, KB, ldo, E;
+  int q_cols;
+  float q_scale;
+  int stages;
+  int bsm_bytes;
+  int tmem_cols;
+  int debug;
+};
+
+struct GemmMisc {
+  uint32_t tmem_base;
+  int abort;
+  int n_tok;
+  int expert;
+  int tokens[kMaxTok];
+  uint32_t touched[kMaxExperts / 32];
+};
+
+template <bool kSwiglu>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid_constant__ GemmArgs a) {
+  constexpr int SUBS = kSwiglu ? 2 : 1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem;
+  uint8_t* bsm = ring + a.stages * kSubBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bsm + a.bsm_bytes);
+  GemmMisc* misc = reinterpret_cast<GemmMisc*>(bars + 2 * a.stages + 2);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8u * a.stages;
+  const uint32_t xready = empty0 + 8u * a.stages;
+  const uint32_t done = xready + 8u;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = gridDim.x;  // split-K factor == cluster size
+  const int rank = static_cast<int>(cluster_rank());
+  const int tile = blockIdx.y;
+  const long long budget = a.debug ? kWaitBudgetDebug : kWaitBudget;
+  volatile int* abort_flag = &misc->abort;
+
+  // ---- which expert and which tokens this CTA serves --------------------------
+  if (a.expert_ids != nullptr) {
+    if (warp == 0) {
+      const int nw = (a.E + 31) >> 5;
+      for (int i = lane; i < nw; i += 32) misc->touched[i] = 0u;
+      __syncwarp();
+      int id0 = lane < a.M ? __ldg(a.expert_ids + lane) : -1;
+      int id1 = lane + 32 < a.M ? __ldg(a.expert_ids + lane + 32) : -1;
+      if ((lane < a.M && (id0 < 0 || id0 >= a.E)) || (lane + 32 < a.M && (id1 < 0 || id1 >= a.E))) {
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) set_status(a.status, kStatusBadExpert);
+      }
+      if (id0 >= a.E) id0 = -1;
+      if (id1 >= a.E) id1 = -1;
+      if (id0 >= 0) atomicOr(&misc->touched[id0 >> 5], 1u << (id0 & 31));
+      if (id1 >= 0) atomicOr(&misc->touched[id1 >> 5], 1u << (id1 & 31));
+      __syncwarp();
+      // the slot-th touched expert, experts in increasing id order
+      const uint32_t word = lane < nw ? misc->touched[lane] : 0u;
+      const int cnt = __popc(word);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = incl - cnt;
+      const int slot = blockIdx.z;
+      int mine = -1;
+      if (slot >= excl && slot < incl) {
+        uint32_t v = word;
+        for (int j = 0; j < slot - excl; ++j) v &= v - 1u;
+        mine = lane * 32 + __ffs(v) - 1;
+      }
+      mine = __reduce_max_sync(0xffffffffu, mine);
+      // this expert's tokens, in token order
+      const unsigned lt = (1u << lane) - 1u;
+      const unsigned b0 = __ballot_sync(0xffffffffu, mine >= 0 && id0 == mine);
+      const unsigned b1 = __ballot_sync(0xffffffffu, mine >= 0 && id1 == mine);
+      if (mine >= 0 && id0 == mine) misc->tokens[__popc(b0 & lt)] = lane;
+      if (mine >= 0 && id1 == mine) misc->tokens[__popc(b0) + __popc(b1 & lt)] = lane + 32;
+      if (lane == 0) {
+        misc->n_tok = mine >= 0 ? __popc(b0) + __popc(b1) : 0;
+        misc->expert = mine >= 0 ? mine : 0;
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    misc->n_tok = a.M;
+    misc->expert = 0;
+  }
+  __syncthreads();
+  const int n_tok = misc->n_tok;
+  const int expert = misc->expert;
+  if (n_tok == 0) return;  // unused expert slot: every CTA of the cluster leaves here
+  const int npad = (n_tok + 7) & ~7;
+  const bool routed = a.expert_ids != nullptr;
+
+  const int kb0 = static_cast<int>(static_cast<long long>(a.KB) * rank / S);
+  const int kb1 = static_cast<int>(static_cast<long long>(a.KB) * (rank + 1) / S);
+  const int nkb = kb1 - kb0;
+  const int nsub = nkb * SUBS;
+  const uint8_t* wsrc = a.w + expert * a.w_expert_bytes +
+                        (static_cast<long long>(tile) * a.KB + kb0) * SUBS * kSubBytes;
+
+  // ---- barriers and Tensor Memory ---------------------------------------------------
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    mbar_init(xready, 64);
+    mbar_init(done, 1);
+    misc->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&misc->tmem_base), static_cast<uint32_t>(a.tmem_cols));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+
+  if (warp == 0) {
+    // ---- weight producer ----
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      const int n_issue = a.debug ? nsub - 1 : nsub;  // test hook: withhold the last stage
+      int issued = 0;
+      for (int i = 0; i < n_issue; ++i) {
+        const int s = i % a.stages;
+        if (i >= a.stages &&
+            !mbar_wait(empty0 + 8u * s, static_cast<uint32_t>((i / a.stages) - 1) & 1u, budget, abort_flag)) {
+          set_status(a.status, kStatusTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(full0 + 8u * s, kSubBytes);
+        bulk_load(smem_u32(ring + s * kSubBytes), wsrc + static_cast<long long>(i) * kSubBytes, kSubBytes,
+                  full0 + 8u * s, pol);
+        issued = i + 1;
+      }
+      if (*abort_flag) {  // let the copies still in flight land before the CTA can exit
+        const int first = issued > a.stages ? issued - a.stages : 0;
+        for (int i = first; i < issued; ++i)
+          mbar_wait(full0 + 8u * (i % a.stages), static_cast<uint32_t>(i / a.stages) & 1u, budget, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      int n_mma = 0;
+      if (!mbar_wait(xready, 0, budget, abort_flag)) {
+        set_status(a.status, kStatusTimeout);
+        *abort_flag = 1;
+      } else {
+        const uint32_t idesc = e4m3_idesc(128, npad);
+        for (int i = 0; i < nsub; ++i) {
+          const int s = i % a.stages;
+          if (!mbar_wait(full0 + 8u * s, static_cast<uint32_t>(i / a.stages) & 1u, budget, abort_flag)) {
+            set_status(a.status, kStatusTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          const int kbl = i / SUBS;
+          const int which = i % SUBS;
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(ring + s * kSubBytes));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(bsm + kbl * npad * 128));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte swizzle row
+            tc_mma_e4m3(tmem + static_cast<uint32_t>(which * npad), adesc + 2u * k, bdesc + 2u * k, idesc,
+                        (kbl > 0 || k > 0) ? 1u : 0u);
+          }
+          ++n_mma;
+          tc_commit(empty0 + 8u * s);  // stage free once these MMAs have read it
+        }
+      }
+      if (n_mma > 0) tc_commit(done);
+      else mbar_arrive(done);
+    }
+    __syncwarp();
+  } else {
+    // ---- activation stager: e4m3 rows -> swizzled K-major B operand ----
+    pdl_wait();  // x_q and s_x are written by the preceding quantise kernel
+    pdl_trigger();
+    const int t = threadIdx.x - 64;
+    const int per_row = nkb * 8;  // 16-byte chunks per token row of this K slice
+    const int chunks = npad * per_row;
+    for (int c = t; c < chunks; c += 64) {
+      const int row = c / per_row;
+      const int rem = c - row * per_row;
+      const int kbl = rem >> 3;
+      const int ch = rem & 7;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < n_tok) {
+        const int tok = routed ? misc->tokens[row] : row;
+        v = *reinterpret_cast<const uint4*>(a.xq + static_cast<long long>(tok) * a.K + (kb0 + kbl) * 128 +
+                                            ch * 16);
+      }
+      uint8_t* dst = bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = v;
+    }
+    fence_async_smem();
+    mbar_arrive(xready);
+  }
+
+  // ---- epilogue: TMEM -> shared partials -> cluster reduction -> bf16 ----------
+  if (!mbar_wait(done, 0, budget, nullptr)) set_status(a.status, kStatusTimeout);
+  tc_fence_after();
+  pdl_wait();
+  fence_async_smem();
+  float* part = reinterpret_cast<float*>(ring);  // [SUBS*npad][128], reuses the drained ring
+  {
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int c0 = 0; c0 < SUBS * npad; c0 += 8) {
+      uint32_t r[8];
+      tmem_ld_x8(lane_base + static_cast<uint32_t>(c0), r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int col = c0 + j;
+        const int m = col % npad;
+        if (m < n_tok) part[col * 128 + row] = __uint_as_float(r[j]);
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // all S partial accumulators are complete and visible
+
+  const float scale = __ldg(a.s_x) * __ldg(a.w_scale + expert);
+  const int r0 = 128 * rank / S;
+  const int rows = 128 * (rank + 1) / S - r0;
+  const int items = rows * n_tok;
+  const uint32_t part_base = smem_u32(part);
+  for (int it = threadIdx.x; it < items; it += kGemmThreads) {
+    const int m = it / rows;
+    const int row = r0 + (it - m * rows);
+    const int tok = routed ? misc->tokens[m] : m;
+    const uint32_t off_g = part_base + static_cast<uint32_t>((m * 128 + row) * 4);
+    float g = 0.0f;
+    float u = 0.0f;
+    for (int p = 0; p < S; ++p) {
+      g += dsmem_ld_f32(dsmem_addr(off_g, p));
+      if (kSwiglu) u += dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p));
+    }
+    if (kSwiglu) {
+      const float yg = g * scale;
+      const float yu = u * scale;
+      const float o = yg / (1.0f + expf(-yg)) * yu;
+      const __nv_bfloat16 b = __float2bfloat16_rn(o);
+      a.out[static_cast<long long>(tok) * a.ldo + tile * 128 + row] = *reinterpret_cast<const uint16_t*>(&b);
+    } else {
+      const int col = tile * 128 + row;
+      float y = g * scale;
+      if (col < a.q_cols) y *= a.q_scale;
+      const __nv_bfloat16 b = __float2bfloat16_rn(y);
+      a.out[static_cast<long long>(tok) * a.ldo + col] = *reinterpret_cast<const uint16_t*>(&b);
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // peers are done reading this CTA's partials
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, static_cast<uint32_t>(a.tmem_cols));
+  }
+}
+
+static int pow2_at_least(int v, int lo) {
+  int p = lo;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
+  const int KB = g.K / 128;
+  const int SUBS = g.swiglu ? 2 : 1;
+  const int n_tiles = g.swiglu ? (g.N / 2) / 128 : g.N / 128;
+  const int npad_max = (g.M + 7) & ~7;
+  const int b_per_kb = npad_max * 128;
+  const int sms = sm_count();
+
+  // split-K: enough CTAs for ~2 per SM, at least enough that each CTA's slice of
+  // the activations fits the B buffer, at most 8 (portable cluster) and KB.
+  int S;
+  if (g.split > 0) {
+    S = g.split;
+  } else {
+    S = (2 * sms) / (n_tiles * g.slots);
+    const int s_fit = (KB * b_per_kb + 45055) / 45056;  // keep B <= 44 KB when possible
+    if (s_fit <= 8 && S < s_fit) S = s_fit;
+  }
+  const int s_min = (KB * b_per_kb + 65535) / 65536;  // hard cap: B <= 64 KB
+  if (S < s_min) S = s_min;
+  if (S < 1) S = 1;
+  if (S > 8) S = 8;
+  if (S > KB) S = KB;
+  if (S < s_min) return cudaErrorInvalidValue;
+  const int nkb_max = (KB + S - 1) / S;
+  const int bsm_bytes = nkb_max * b_per_kb;
+  const int part_bytes = SUBS * npad_max * 128 * 4;
+  const int misc_bytes = static_cast<int>(sizeof(GemmMisc));
+  auto smem_for = [&](int st) { return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 2) * 8 + misc_bytes; };
+  int stages = 6;
+  if (2 * (smem_for(6) + 1024) > 233472) stages = 4;
+  if (2 * (smem_for(4) + 1024) > 233472) stages = 6;  // one CTA per SM: keep the deep ring
+  while (stages * kSubBytes < part_bytes) ++stages;
+  int smem = smem_for(stages);
+  if (smem > 232448) return cudaErrorInvalidValue;
+  const int tmem_cols = pow2_at_least(SUBS * npad_max, 32);
+  // TMEM safety: the CTAs that can share an SM must fit in its 512 columns.
+  while ((233472 / (smem + 1024)) * tmem_cols > 512) smem += 1024;
+
+  GemmArgs a;
+  a.w = g.w;
+  a.w_expert_bytes = g.w_expert_bytes;
+  a.w_scale = g.w_scale;
+  a.xq = g.xq;
+  a.s_x = g.s_x;
+  a.status = g.status;
+  a.out = g.out;
+  a.expert_ids = g.expert_ids;
+  a.M = g.M;
+  a.K = g.K;
+  a.KB = KB;
+  a.ldo = g.ldo;
+  a.E = g.E;
+  a.q_cols = g.q_cols;
+  a.q_scale = g.q_scale;
+  a.stages = stages;
+  a.bsm_bytes = bsm_bytes;
+  a.tmem_cols = tmem_cols;
+  a.debug = g.debug ? 1 : 0;
+
+  Launch L(dim3(S, n_tiles, g.slots), dim3(kGemmThreads), static_cast<size_t>(smem), s,
+           static_cast<unsigned>(S), g.pdl);
+  cudaError_t e;
+  if (g.swiglu) {
+    e = cudaFuncSetAttribute(gemm_e4m3_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&L.cfg, gemm_e4m3_kernel<true>, a);
+  }
+  e = cudaFuncSetAttribute(gemm_e4m3_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&L.cfg, gemm_e4m3_kernel<false>, a);
+}
+
+}  // namespace dl
