@@ -61,7 +61,7 @@ def run_qkv(x, w, s_w, Hq, Hkv, d, q_scale, flags=dl.DL_FLAG_PDL, split=0):
 def test_pack_matches_stated_layout(N, K, kind):
     g = np.random.default_rng(N + K + kind)
     w = g.integers(0, 256, size=(N, K)).astype(np.uint8)
-    got = pack(w, kind).cpu().numpy()
+    got = pack(w, kind).cpu().numpy().ravel()
     assert np.array_equal(got, helpers.pack_reference(w, kind))
 
 
