@@ -20,9 +20,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,8 +34,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="layer_b1")
     p.add_argument("--cluster", type=int, default=0, help="attention cluster size (0 = workload default)")
@@ -121,51 +119,66 @@ def run_reference(args):
 # --------------------------------------------------------------- clocks --------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    through NVML from a background thread (~1 kHz), so that even a
+    sub-second timed region gets samples.  Read-only: changes no setting."""
 
-    def __init__(self, device_index):
-        self.dev = device_index
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, torch_device_index):
+        self.idx = torch_device_index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
+        self._handle = None
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(self.idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+            self._nvml = pynvml
+        except Exception:  # NVML unavailable: report "unsampled"
+            self._nvml = None
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            nv, h = self._nvml, self._handle
+            bits = {k: getattr(nv, v) for k, v in self.REASONS.items()}
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for k, b in bits.items():
+                        if r & b:
+                            self.reasons.add(k)
+                except Exception:
+                    pass
+                time.sleep(0.001)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for i, n in enumerate(names):
-                if r[5 + i].lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(rows)}
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=5)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------- GPU arm --------
@@ -245,8 +258,10 @@ def run_ours(args):
     h = stream.cuda_stream
 
     def step(i, flags=dl.DL_FLAG_PDL):
+        # launch on torch's current stream: the eager stream, or the capturing one inside a graph capture
         r = i % R
-        layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens, stream=h, flags=flags)
+        layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens,
+                       stream=torch.cuda.current_stream().cuda_stream, flags=flags)
 
     for i in range(max(args.warmup, 3)):
         step(i)
@@ -258,11 +273,56 @@ def run_ours(args):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    # ---- timed region: K whole-layer steps ----
+    # ---- CUDA graphs of the PDL-chained steps (the launch mode the pages pair with PDL) ----
+    cap_stream = torch.cuda.Stream(device)
+
+    def capture(fn, idxs):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            for i in idxs:
+                fn(i)
+        return g
+
+    G = R * max(1, 24 // R)
+    graphs = None
+    try:
+        graphs = (capture(step, range(G)), [capture(step, [r]) for r in range(R)])
+    except Exception as exc:  # capture refused: fall back to direct launches, and say so
+        graphs = None
+        graph_error = repr(exc)[:200]
+    torch.cuda.synchronize()
+
+    def graph_steps(n, big, singles, period):
+        q, rem = divmod(n, period)
+        for _ in range(q):
+            big.replay()
+        for j in range(rem):
+            singles[(q * period + j) % len(singles)].replay()
+
+    def timed_graph(n, big, singles, period):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record()
+        graph_steps(n, big, singles, period)
+        end.record()
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    if graphs is not None:
+        for _ in range(2):
+            graph_steps(max(args.warmup, 3), graphs[0], graphs[1], G)
+
+    # ---- timed region: exactly K whole-layer steps ----
     clocks = ClockSampler(local)
     barrier()
     clocks.start()
-    ms = timed(step, args.steps, stream)
+    if graphs is not None:
+        ms = timed_graph(args.steps, graphs[0], graphs[1], G)
+        launch_mode = f"CUDA graph of {G} PDL-chained layer steps, replayed"
+    else:
+        ms = timed(step, args.steps, stream)
+        launch_mode = "direct launches (graph capture failed: " + graph_error + ")"
     barrier()
     clk = clocks.stop()
     for lay in layers:
@@ -272,8 +332,16 @@ def run_ours(args):
         t = torch.tensor([us_layer], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         us_layer = float(t.item())
+    layer_bytes = wl.n_qkv * wl.K + wl.N2 * wl.K + int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
+    if layer_bytes / (us_layer * 1e-6) / 1e9 > 1.2 * peak_hbm()[0]:
+        raise SystemExit(f"timed region did not do the work: {us_layer:.3f} us per layer is faster than HBM allows")
 
-    # ---- the same steps without PDL (context) ----
+    # ---- context: direct launches through the public API (PDL on / off), host time per step ----
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ms_direct = timed(step, args.steps, stream)
+    host_us = (time.perf_counter() - t0) * 1e6 / args.steps
+    us_layer_direct = ms_direct * 1e3 / args.steps
     us_layer_nopdl = timed(lambda i: step(i, 0), args.steps, stream) * 1e3 / args.steps
 
     # ---- per-call loops, for the roofline of each kernel family ----
@@ -282,18 +350,20 @@ def run_ours(args):
         r = i % R
         L_ = layers[r]
         dl.check(dl.dl_fc_qkv_scale(xs[r][0], wl.M, K, L_.wp_qkv, L_.s_qkv, wl.Hq, wl.Hkv, wl.d, L_.q_scale, L_.qkv,
-                                    L_.ws_qkv, stream=h))
+                                    L_.ws_qkv, stream=torch.cuda.current_stream().cuda_stream))
 
     def call_attn(i):
         r = i % R
         L_ = layers[r]
         dl.check(dl.dl_decode_attn(L_.qkv, L_.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, kvs[r][0], kvs[r][1],
-                                   wl.Lcap, seq_lens, 1.0, cluster, L_.attn_out, L_.ws_attn, stream=h))
+                                   wl.Lcap, seq_lens, 1.0, cluster, L_.attn_out, L_.ws_attn,
+                                   stream=torch.cuda.current_stream().cuda_stream))
 
     def call_fc13(i):
         r = i % R
         L_ = layers[r]
-        dl.check(dl.dl_fc13_swiglu(xs[r][1], wl.M, K, L_.wp_13, L_.s_13, wl.N2, L_.ffn_out, L_.ws_13, stream=h))
+        dl.check(dl.dl_fc13_swiglu(xs[r][1], wl.M, K, L_.wp_13, L_.s_13, wl.N2, L_.ffn_out, L_.ws_13,
+                                   stream=torch.cuda.current_stream().cuda_stream))
 
     kv_bytes = int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
     fam = {
@@ -306,10 +376,17 @@ def run_ours(args):
     for name, (fn, nbytes, launches) in fam.items():
         for i in range(3):
             fn(i)
-        us = timed(fn, args.steps, stream) * 1e3 / args.steps
+        mode = "direct"
+        try:
+            gbig, gs = capture(fn, range(G)), [capture(fn, [r]) for r in range(R)]
+            graph_steps(6, gbig, gs, G)
+            us = timed_graph(args.steps, gbig, gs, G) * 1e3 / args.steps
+            mode = "graph"
+        except Exception:
+            us = timed(fn, args.steps, stream) * 1e3 / args.steps
         gbs = nbytes / (us * 1e-6) / 1e9
         kernels[name] = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak,
-                         "launches_per_call": launches}
+                         "launches_per_call": launches, "mode": mode}
     for lay in layers:
         lay.read_status(h)
 
@@ -365,7 +442,10 @@ def run_ours(args):
                      "achieved": dom["achieved_gbs"], "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": dom["achieved_gbs"] / peak, "traffic": None},
         "kernels": kernels,
-        "layer_us_no_pdl": us_layer_nopdl,
+        "layer_us_direct_launch": us_layer_direct,
+        "layer_us_direct_no_pdl": us_layer_nopdl,
+        "host_us_per_step_direct": host_us,
+        "launch": launch_mode,
         "layer_alg_bytes": wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes,
         "layer_achieved_gbs": (wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes) / (us_layer * 1e-6) / 1e9,
         "e2e": {"value": us_e2e, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
