@@ -124,6 +124,35 @@ dl_status dl_fc13_swiglu(const uint16_t* x, int M, int K, const uint8_t* w_packe
                          size_t ws_bytes, void* stream, unsigned flags);
 
 /* ---------------------------------------------------------------------------
+ * FC13 + SwiGLU without a caller workspace.  The source pages have no
+ * counterpart of this entry point; it exists for callers that cannot allocate
+ * device memory: a plugin that its host runtime hands only input and output
+ * buffers, an engine that reserves its whole memory pool at start-up and
+ * forbids later allocations, or a latency-critical loop where cudaMalloc or
+ * cudaFree would synchronise the device.
+ *
+ * Same computation, arguments and requirements as dl_fc13_swiglu, except:
+ *   - the activation scratch (e4m3 x_q and s_x) lives in one fixed device
+ *     array inside libdl.so of 256 + 64*8192 bytes, held by every GPU that
+ *     loads the library until the process exits.  M > 64 or M*K > 64*8192
+ *     returns DL_ERR_WORKSPACE before anything is launched.
+ *   - `status` is an optional device uint32 that the caller zeroes; device-
+ *     side errors (bit 1 timeout) are OR-ed into it.  NULL: not reported.
+ *   - nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *     library routine is called.
+ *   - the first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress, once per device, with that device current);
+ *     make that first call before any stream capture.
+ *   - every call shares the array and leaves its contents behind; calls that
+ *     overlap on the GPU (concurrent streams or unordered host threads) race
+ *     on it.  Calls queued in order on one stream, with or without
+ *     DL_FLAG_PDL, are safe.
+ * ------------------------------------------------------------------------- */
+dl_status dl_fc13_swiglu_static_ws(const uint16_t* x, int M, int K, const uint8_t* w_packed,
+                                   const float* w_scale, int N2, uint16_t* out, uint32_t* status,
+                                   void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
  * FC_QKV + attention scaling.  [XZY] "运算融合"; [NV] fusion list.
  *   w_packed e4m3, DL_PACK_PLAIN layout of the [(Hq+2*Hkv)*d][K] weight
  *   qkv     bf16 [M][(Hq+2*Hkv)*d], row-major: Q heads, then K heads, then V heads

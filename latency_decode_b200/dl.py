@@ -44,6 +44,7 @@ _SIGNATURES = {
     "dl_pack_fp8_weight": (_I, [_P, _P, _I, _I, _I, _P]),
     "dl_workspace_bytes": (_SZ, [_I, _I]),
     "dl_fc13_swiglu": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
+    "dl_fc13_swiglu_static_ws": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _P, _U]),
     "dl_fc_qkv_scale": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P, _SZ, _P, _U]),
     "dl_moe_fc13_swiglu_grouped": (_I, [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
     "dl_decode_attn": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
@@ -115,6 +116,12 @@ def dl_fc13_swiglu(x, M, K, w_packed, w_scale, N2, out, ws, ws_bytes=None, strea
                    flags=DL_FLAG_PDL) -> int:
     return lib().dl_fc13_swiglu(_ptr(x), M, K, _ptr(w_packed), _ptr(w_scale), N2, _ptr(out), _ptr(ws),
                                 _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_fc13_swiglu_static_ws(x, M, K, w_packed, w_scale, N2, out, status=None, stream=None,
+                             flags=DL_FLAG_PDL) -> int:
+    return lib().dl_fc13_swiglu_static_ws(_ptr(x), M, K, _ptr(w_packed), _ptr(w_scale), N2, _ptr(out),
+                                          _ptr(status), _stream(stream), flags)
 
 
 def dl_fc_qkv_scale(x, M, K, w_packed, w_scale, Hq, Hkv, d, q_scale, qkv, ws, ws_bytes=None,
