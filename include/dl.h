@@ -72,7 +72,9 @@ typedef enum dl_status {
                                      withholds the last pipeline load, so the consumer's
                                      wait runs out and DL_ERR_TIMEOUT is reported */
 #define DL_FLAG_SPLIT_SHIFT 8     /* bits [8,13): if non-zero, force the GEMM split-K
-                                     cluster size (1..8) instead of the built-in choice */
+                                     cluster size (1..8), or the number of clusters per
+                                     (b, kv head) of dl_decode_attn (1..16), instead of
+                                     the built-in choice */
 
 /* weight pack kinds */
 #define DL_PACK_PLAIN 0   /* FC_QKV and other plain projections */
@@ -103,8 +105,9 @@ dl_status dl_pack_fp8_weight(const uint8_t* w_nk, uint8_t* w_packed, int N, int 
                              void* stream);
 
 /* Bytes of workspace a GEMM call with M rows of K activations needs
- * (256 + M*K rounded up to 256).  dl_workspace_bytes(0, 0) = 256 is what
- * dl_decode_attn needs (the status word only). */
+ * (256 + M*K rounded up to 256).  dl_workspace_bytes(0, 0) = 256 (the status
+ * word only) is the least dl_decode_attn accepts; see
+ * dl_decode_attn_workspace_bytes for the size it can use. */
 size_t dl_workspace_bytes(int M, int K);
 
 /* ---------------------------------------------------------------------------
@@ -205,6 +208,12 @@ dl_status dl_moe_fc13_swiglu_grouped(const uint16_t* x, int T, int K, const int3
  * head h / (Hq/Hkv).  Each (b, kv head) is handled by one cluster of
  * cluster_size CTAs (1, 2, 4, 8 or 16); CTA r streams the r-th contiguous
  * chunk of ceil(L/cluster_size) keys (rounded up to 16).
+ * When the workspace allows (dl_decode_attn_workspace_bytes), each (b, kv
+ * head) may be split over several clusters of cluster_size CTAs; their
+ * DSMEM-merged states are merged once more through the workspace.  The
+ * DL_FLAG_SPLIT_SHIFT bits, when non-zero, force that number of clusters
+ * (1..16).  ws must be zero-filled before its first use; every call leaves
+ * its counters at zero again.
  * Supported: d in {64, 128}, Hq % Hkv == 0, (Hq/Hkv)*T <= 32, q_token_stride
  * a multiple of 8 and >= Hq*d.
  * ------------------------------------------------------------------------- */
@@ -213,6 +222,16 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
                          int Lcap, const int32_t* seq_lens, float softmax_scale,
                          int cluster_size, uint16_t* out, void* ws, size_t ws_bytes,
                          void* stream, unsigned flags);
+
+/* Workspace bytes for dl_decode_attn at these shapes.  When B*Hkv*cluster_size
+ * CTAs would leave the GPU half idle, dl_decode_attn splits each (b, kv head)
+ * over several clusters whose merged states meet in the workspace (the last
+ * cluster to finish merges them and resets its counter); this returns the size
+ * that allows the built-in choice.  A smaller workspace (down to 256 bytes)
+ * is accepted and simply allows fewer clusters per head.  Returns 0 for
+ * invalid shapes. */
+size_t dl_decode_attn_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Lcap,
+                                      int cluster_size);
 
 /* Synchronises `stream`, reads the status word of `ws`, clears it, and returns
  * DL_OK, DL_ERR_TIMEOUT or DL_ERR_DEVICE_ARG (timeout takes precedence). */

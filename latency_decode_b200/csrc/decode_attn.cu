@@ -8,10 +8,11 @@
 // optimisation and fusion" (same two points).
 //
 // Design (B200-native; the pages give no code):
-//  * one cluster of S CTAs per (sequence b, kv head); CTA r streams the r-th
-//    contiguous chunk of ceil(L/S) keys (rounded up to 16).  The G = Hq/Hkv
-//    query heads of the group and the T query tokens share every K/V byte
-//    loaded, so K and V are read exactly once.
+//  * the keys of one (sequence b, kv head) are split into P*S contiguous
+//    chunks of ceil(L/(P*S)) keys (rounded up to 16), one per CTA; the S CTAs
+//    of a thread-block cluster hold S neighbouring chunks.  The G = Hq/Hkv query
+//    heads and the T query tokens share every K/V byte loaded, so K and V are
+//    read exactly once.
 //  * a producer warp moves 64-key tiles of K and V with TMA tensor copies in the
 //    128-byte swizzle (bank-conflict-free ldmatrix), into a ring of stages; it
 //    does not wait for the preceding kernel (the KV cache is static), so under
@@ -19,11 +20,17 @@
 //  * four consumer warps each take 16 keys of a tile and run swapped-AB
 //    tensor-core MMAs (mma.sync m16n8k16, bf16 -> fp32): S^T = K Q^T with the
 //    keys as the M dimension and the R = G*T query rows as N (padded to 8, not
-//    16), then O^T += V^T P^T.  P^T is formed in registers with movmatrix.
+//    16), then O^T += V^T P^T.  P^T is formed in registers with movmatrix; the
+//    Q^T fragments are read from shared memory, which keeps two CTAs per SM.
 //  * online softmax in the log2 domain; the row max is a 3-step warp shuffle.
-//  * the four warp states merge in shared memory, then the S CTA states merge
-//    through distributed shared memory: M* = max m_i, L* = sum l_i 2^(m_i-M*),
-//    o = sum o_i 2^(m_i-M*) / L*; each CTA finalises 1/S of the outputs.
+//  * merges: the four warp states merge in shared memory; the S CTA states of
+//    a cluster merge through distributed shared memory (M* = max m_i,
+//    L* = sum l_i 2^(m_i-M*), o = sum o_i 2^(m_i-M*) / L*), each CTA owning
+//    1/S of the outputs.  With P = 1 that is the final result.  With P > 1
+//    (used when B*Hkv*S CTAs would leave the GPU half idle) each cluster
+//    stores its merged state in the workspace and bumps a per-(b, kv head)
+//    counter; the cluster that arrives last merges the P states the same way
+//    and resets the counter.  Nothing ever waits for another cluster.
 #include <cudaTypedefs.h>
 
 #include "dl_device.cuh"
@@ -34,6 +41,7 @@ namespace dl {
 constexpr int kAttnKT = 64;           // keys per pipeline stage
 constexpr int kAttnConsumers = 4;     // consumer warps, 16 keys each per stage
 constexpr int kAttnThreads = 32 * (kAttnConsumers + 1);
+constexpr int kAttnMaxSplits = 16;    // clusters per (b, kv head)
 
 struct AttnArgs {
   const uint16_t* q;
@@ -43,6 +51,11 @@ struct AttnArgs {
   float scale_log2;  // softmax scale * log2(e)
   uint16_t* out;
   uint32_t* status;
+  uint32_t* counters;  // [B*Hkv], P > 1 only
+  float* part_m;       // [B*Hkv][P][R]
+  float* part_l;       // [B*Hkv][P][R]
+  float* part_o;       // [B*Hkv][P][R][D]
+  int P;
   int stages;
   int debug;
 };
@@ -52,7 +65,7 @@ __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
 }
 
 template <int D, int NT>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ AttnArgs a) {
   constexpr int HALVES = D / 64;              // a swizzled row holds 64 bf16 (128 bytes)
@@ -63,8 +76,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + a.stages * STAGE_BYTES);
+  uint2* qs = reinterpret_cast<uint2*>(ring + a.stages * STAGE_BYTES);        // [KS][NT][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qs + KS * NT * 32);
   int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages);
+  int* last_word = abort_word + 1;
   volatile int* abort_flag = abort_word;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8u * a.stages;
@@ -74,17 +89,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int S = gridDim.x;
   const int rank = static_cast<int>(cluster_rank());
   const int hk = blockIdx.y;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z / a.P;
+  const int split = blockIdx.z - b * a.P;
   const long long budget = a.debug ? kWaitBudgetDebug : kWaitBudget;
 
   // ---- this CTA's key chunk ----
   int L = __ldg(a.seq_lens + b);
   if (L < a.T || L > a.Lcap) {
-    if (threadIdx.x == 0 && rank == 0 && hk == 0) set_status(a.status, kStatusBadSeqLen);
+    if (threadIdx.x == 0 && rank == 0 && hk == 0 && split == 0) set_status(a.status, kStatusBadSeqLen);
     L = 0;  // no visible keys: the output of this sequence is zero
   }
-  const int chunk = (((L + S - 1) / S) + 15) & ~15;
-  const int lo = min(rank * chunk, L);
+  const int nchunks = a.P * S;
+  const int chunk = (((L + nchunks - 1) / nchunks) + 15) & ~15;
+  const int lo = min((split * S + rank) * chunk, L);
   const int hi = min(lo + chunk, L);
   const int n_tiles = (hi - lo + kAttnKT - 1) / kAttnKT;
 
@@ -94,6 +111,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(empty0 + 8u * s, kAttnConsumers);
     }
     *abort_word = 0;
+    *last_word = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -157,27 +175,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     pdl_wait();  // q is written by the preceding QKV GEMM
     if (threadIdx.x == 0) pdl_trigger();
 
-    // Q^T fragments (B operand of S^T = K Q^T): column n = query row g of tile nt
-    uint32_t qf[KS][NT][2];
+    // Q^T fragments (B operand of S^T = K Q^T), column n = query row g of tile nt,
+    // staged once in shared memory by the four consumer warps.
+    for (int f = threadIdx.x; f < KS * NT * 32; f += 32 * kAttnConsumers) {
+      const int ln = f & 31;
+      const int nt = (f >> 5) % NT;
+      const int ks = (f >> 5) / NT;
+      const int rho = nt * 8 + (ln >> 2);
+      uint2 v = make_uint2(0u, 0u);
+      if (rho < a.R) {
+        const int t = rho / a.G;
+        const int hq = hk * a.G + rho % a.G;
+        const uint16_t* qrow =
+            a.q + (static_cast<long long>(b) * a.T + t) * a.q_stride + static_cast<long long>(hq) * D;
+        v.x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
+        v.y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
+      }
+      qs[f] = v;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kAttnConsumers) : "memory");
+
     int lim[NT][2];  // last visible key of the rows this thread accumulates
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int rho = nt * 8 + g;
-      const bool valid = rho < a.R;
-      const int t = valid ? rho / a.G : 0;
-      const int hq = hk * a.G + (valid ? rho % a.G : 0);
-      const uint16_t* qrow = a.q + (static_cast<long long>(b) * a.T + t) * a.q_stride + static_cast<long long>(hq) * D;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qf[ks][nt][0] = valid ? ld_b32(qrow + ks * 16 + 2 * q4) : 0u;
-        qf[ks][nt][1] = valid ? ld_b32(qrow + ks * 16 + 8 + 2 * q4) : 0u;
-      }
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int r2 = nt * 8 + 2 * q4 + j;
         lim[nt][j] = r2 < a.R ? L - a.T + r2 / a.G : -1;
       }
-    }
 
     for (int i = 0; i < n_tiles; ++i) {
       const int s = i % a.stages;
@@ -209,7 +234,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint2 qf = qs[(ks * NT + nt) * 32 + lane];
+              mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
+            }
           }
         }
         // ---- online softmax (log2 domain) ----
@@ -330,41 +358,109 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   cluster_sync();  // every CTA state of the cluster is visible through DSMEM
 
-  // ---- merge the S CTA states; CTA `rank` finalises a 1/S slice of the outputs ----
+  // ---- merge the S CTA states; CTA `rank` handles a 1/S slice of the outputs ----
   const int items = R * (D / 4);
   const int i0 = static_cast<int>(static_cast<long long>(items) * rank / S);
   const int i1 = static_cast<int>(static_cast<long long>(items) * (rank + 1) / S);
   const uint32_t cm_l = smem_u32(cm), cl_l = smem_u32(cl), co_l = smem_u32(co);
+  const long long head = static_cast<long long>(b) * a.Hkv + hk;
   for (int it = i0 + threadIdx.x; it < i1; it += kAttnThreads) {
     const int rho = it / (D / 4);
     const int c4 = it - rho * (D / 4);
-    float M = -INFINITY;
-    for (int p = 0; p < S; ++p) {
-      const float lp = dsmem_ld_f32(dsmem_addr(cl_l + 4u * rho, p));
-      if (lp > 0.0f) M = fmaxf(M, dsmem_ld_f32(dsmem_addr(cm_l + 4u * rho, p)));
+    float mp[16], lp[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {  // issue every peer load before using them
+      if (p < S) {
+        lp[p] = dsmem_ld_f32(dsmem_addr(cl_l + 4u * rho, p));
+        mp[p] = dsmem_ld_f32(dsmem_addr(cm_l + 4u * rho, p));
+      }
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+      if (p < S && lp[p] > 0.0f) M = fmaxf(M, mp[p]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.0f;
-    for (int p = 0; p < S; ++p) {
-      const float lp = dsmem_ld_f32(dsmem_addr(cl_l + 4u * rho, p));
-      if (lp > 0.0f) {
-        const float f = ex2(dsmem_ld_f32(dsmem_addr(cm_l + 4u * rho, p)) - M);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      if (p < S && lp[p] > 0.0f) {
+        const float f = ex2(mp[p] - M);
         const float4 v = dsmem_ld_f32x4(dsmem_addr(co_l + 4u * (rho * D + c4 * 4), p));
         acc.x += v.x * f;
         acc.y += v.y * f;
         acc.z += v.z * f;
         acc.w += v.w * f;
-        lsum += lp * f;
+        lsum += lp[p] * f;
       }
     }
-    const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-    const int t = rho / a.G;
-    const int hq = hk * a.G + rho % a.G;
-    uint16_t* dst = a.out + ((static_cast<long long>(b) * a.T + t) * a.Hq + hq) * D + c4 * 4;
-    uint2 packed;
-    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(dst) = packed;
+    if (a.P == 1) {
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      const int t = rho / a.G;
+      const int hq = hk * a.G + rho % a.G;
+      uint16_t* dst = a.out + ((static_cast<long long>(b) * a.T + t) * a.Hq + hq) * D + c4 * 4;
+      uint2 packed;
+      packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(dst) = packed;
+    } else {
+      // this cluster's merged state, unnormalised, for the cross-cluster merge
+      const long long slot = head * a.P + split;
+      *reinterpret_cast<float4*>(a.part_o + (slot * R + rho) * D + c4 * 4) = acc;
+      if (c4 == 0) {
+        a.part_m[slot * R + rho] = M;
+        a.part_l[slot * R + rho] = lsum;
+      }
+    }
+  }
+  if (a.P > 1) {
+    __threadfence();
+    cluster_sync();  // every CTA of this cluster has stored and fenced its slice
+    if (rank == 0 && threadIdx.x == 0) {
+      const unsigned prev = atomicAdd(a.counters + head, 1u);
+      const int last = prev == static_cast<unsigned>(a.P - 1);
+      if (last) {
+        __threadfence();
+        a.counters[head] = 0u;  // every other cluster of this head has arrived: reset for the next call
+      }
+      *last_word = last;
+    }
+    cluster_sync();
+    const int last = static_cast<int>(dsmem_ld_u32(dsmem_addr(smem_u32(last_word), 0)));
+    if (last) {
+      __threadfence();
+      for (int it = i0 + threadIdx.x; it < i1; it += kAttnThreads) {
+        const int rho = it / (D / 4);
+        const int c4 = it - rho * (D / 4);
+        float M = -INFINITY;
+        for (int p = 0; p < a.P; ++p) {
+          const long long slot = head * a.P + p;
+          if (__ldcg(a.part_l + slot * R + rho) > 0.0f) M = fmaxf(M, __ldcg(a.part_m + slot * R + rho));
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lsum = 0.0f;
+        for (int p = 0; p < a.P; ++p) {
+          const long long slot = head * a.P + p;
+          const float lq = __ldcg(a.part_l + slot * R + rho);
+          if (lq > 0.0f) {
+            const float f = ex2(__ldcg(a.part_m + slot * R + rho) - M);
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (slot * R + rho) * D + c4 * 4));
+            acc.x += v.x * f;
+            acc.y += v.y * f;
+            acc.z += v.z * f;
+            acc.w += v.w * f;
+            lsum += lq * f;
+          }
+        }
+        const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+        const int t = rho / a.G;
+        const int hq = hk * a.G + rho % a.G;
+        uint16_t* dst = a.out + ((static_cast<long long>(b) * a.T + t) * a.Hq + hq) * D + c4 * 4;
+        uint2 packed;
+        packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(dst) = packed;
+      }
+    }
   }
   cluster_sync();  // keep this CTA's state alive until every peer has read it
 }
@@ -396,17 +492,39 @@ static bool encode_kv_map(CUtensorMap* m, const uint16_t* base, int d, int Lcap,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Workspace of dl_decode_attn with P clusters per (b, kv head): the 256-byte
+// header, then the per-head counters, then the P cluster states.
+size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P) {
+  if (P <= 1) return kWsHeader;
+  const size_t heads = static_cast<size_t>(B) * Hkv;
+  const size_t counters = (heads * 4 + 255) / 256 * 256;
+  const size_t ml = (heads * P * R * 4 + 255) / 256 * 256;
+  return kWsHeader + counters + 2 * ml + heads * P * R * d * 4;
+}
+
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap) {
+  const long long base = static_cast<long long>(B) * Hkv * cluster;
+  const long long target = 2ll * sm_count();  // two CTAs per SM
+  if (base >= target) return 1;
+  long long P = target / base;
+  const long long by_len = Lcap / (static_cast<long long>(cluster) * 2 * kAttnKT);  // >= 2 tiles per CTA
+  if (P > by_len) P = by_len;
+  if (P > kAttnMaxSplits) P = kAttnMaxSplits;
+  return P < 1 ? 1 : static_cast<int>(P);
+}
+
 template <int D, int NT>
 static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                                  const AttnLaunch& p, cudaStream_t s) {
   constexpr int STAGE_BYTES = 2 * (D / 64) * kAttnKT * 128;
   const int R = a.R;
   const int merge_bytes = (kAttnConsumers * R * D + 2 * kAttnConsumers * R + 2 * R + 4 + R * D) * 4;
-  int stages = a.stages;
+  int stages = D == 128 ? 3 : 6;  // ~100 KB of ring: two CTAs per SM
   while (stages * STAGE_BYTES < merge_bytes) ++stages;
   AttnArgs args = a;
   args.stages = stages;
-  const int smem = 1024 + stages * STAGE_BYTES + 2 * stages * 8 + 16;
+  const int qs_bytes = (D / 16) * NT * 32 * 8;
+  const int smem = 1024 + stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16;
   auto kern = decode_attn_kernel<D, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -414,7 +532,7 @@ static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, c
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  Launch L(dim3(p.cluster, p.Hkv, p.B), dim3(kAttnThreads), static_cast<size_t>(smem), s,
+  Launch L(dim3(p.cluster, p.Hkv, p.B * a.P), dim3(kAttnThreads), static_cast<size_t>(smem), s,
            static_cast<unsigned>(p.cluster), p.pdl);
   return cudaLaunchKernelEx(&L.cfg, kern, tk, tv, args);
 }
@@ -437,8 +555,25 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.out = p.out;
   a.status = p.status;
-  a.stages = 4;
+  a.stages = 3;
   a.debug = p.debug ? 1 : 0;
+  // clusters per (b, kv head): forced, else automatic; then as many as the workspace holds
+  int P = p.splits > 0 ? p.splits : attn_auto_splits(p.B, p.Hkv, p.cluster, p.Lcap);
+  while (P > 1 && attn_ws_bytes(p.B, p.Hkv, a.R, p.d, P) > p.ws_bytes) --P;
+  if (static_cast<long long>(p.B) * P > 65535) P = 1;
+  a.P = P;
+  a.counters = nullptr;
+  a.part_m = a.part_l = a.part_o = nullptr;
+  if (P > 1) {
+    const size_t heads = static_cast<size_t>(p.B) * p.Hkv;
+    uint8_t* base = reinterpret_cast<uint8_t*>(p.status) + kWsHeader;
+    a.counters = reinterpret_cast<uint32_t*>(base);
+    base += (heads * 4 + 255) / 256 * 256;
+    const size_t ml = (heads * P * a.R * 4 + 255) / 256 * 256;
+    a.part_m = reinterpret_cast<float*>(base);
+    a.part_l = reinterpret_cast<float*>(base + ml);
+    a.part_o = reinterpret_cast<float*>(base + 2 * ml);
+  }
   const int NT = (a.R + 7) / 8;
   if (p.d == 128) {
     switch (NT) {

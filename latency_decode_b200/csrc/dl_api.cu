@@ -59,6 +59,12 @@ size_t dl_workspace_bytes(int M, int K) {
   return dl::kWsHeader + ((q + 255) / 256) * 256;
 }
 
+size_t dl_decode_attn_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Lcap, int cluster_size) {
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || d < 1 || Lcap < 1 || cluster_size < 1 || Hq % Hkv != 0) return 0;
+  const int P = dl::attn_auto_splits(B, Hkv, cluster_size, Lcap);
+  return dl::attn_ws_bytes(B, Hkv, (Hq / Hkv) * T, d, P);
+}
+
 dl_status dl_pack_fp8_weight(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
                              void* stream) {
   if (w_nk == nullptr || w_packed == nullptr || N < 1 || K < 1) return DL_ERR_INVALID_ARG;
@@ -77,9 +83,15 @@ static dl_status run_dense_gemm(const uint16_t* x, int M, int K, const uint8_t* 
                                 void* stream, unsigned flags) {
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool pdl = (flags & DL_FLAG_PDL) != 0;
-  cudaError_t e = dl::launch_act_quant(x, M, K, dl::ws_xq(ws), dl::ws_sx(ws), s, pdl);
-  if (e != cudaSuccess) return cuda_status(e);
+  // Small inputs are quantised inside the GEMM (one launch); larger ones by the
+  // cluster quantise kernel first.  Both write x_q and s_x to the workspace.
+  const bool fused = static_cast<long long>(M) * K <= dl::kFusedQuantMaxElems;
+  if (!fused) {
+    cudaError_t e = dl::launch_act_quant(x, M, K, dl::ws_xq(ws), dl::ws_sx(ws), s, pdl);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   dl::GemmLaunch g{};
+  g.x = fused ? x : nullptr;
   g.w = w_packed;
   g.w_expert_bytes = 0;
   g.w_scale = w_scale;
@@ -183,6 +195,7 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
   if (cluster_size != 1 && cluster_size != 2 && cluster_size != 4 && cluster_size != 8 && cluster_size != 16)
     return DL_ERR_INVALID_ARG;
   if (q_token_stride < static_cast<long long>(Hq) * d || q_token_stride % 8 != 0) return DL_ERR_ALIGNMENT;
+  if (forced_split(flags) > 16) return DL_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
       !aligned(seq_lens, 4))
     return DL_ERR_ALIGNMENT;
@@ -202,6 +215,8 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
   a.seq_lens = seq_lens;
   a.scale = softmax_scale;
   a.cluster = cluster_size;
+  a.splits = static_cast<int>(forced_split(flags));
+  a.ws_bytes = ws_bytes;
   a.out = out;
   a.status = dl::ws_status(ws);
   a.debug = (flags & DL_FLAG_DEBUG_TIMEOUT) != 0;

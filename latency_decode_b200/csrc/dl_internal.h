@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/dl.h"
+#include "dl.h"
 
 namespace dl {
 
@@ -54,8 +54,9 @@ struct GemmLaunch {
   const uint8_t* w;
   long long w_expert_bytes;
   const float* w_scale;
-  const uint8_t* xq;
-  const float* s_x;
+  uint8_t* xq;
+  float* s_x;
+  const uint16_t* x;          // non-null: quantise x inside the GEMM (dense, small M*K)
   uint32_t* status;
   uint16_t* out;
   const int32_t* expert_ids;  // null for dense
@@ -69,6 +70,8 @@ struct GemmLaunch {
   bool pdl;
 };
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s);
+// Largest M*K for which a dense GEMM quantises its activations itself.
+constexpr long long kFusedQuantMaxElems = 32768;
 
 struct AttnLaunch {
   const uint16_t* q;
@@ -79,11 +82,15 @@ struct AttnLaunch {
   const int32_t* seq_lens;
   float scale;
   int cluster;
+  int splits;        // clusters per (b, kv head); 0 = automatic
+  size_t ws_bytes;   // workspace available (limits the number of clusters per head)
   uint16_t* out;
-  uint32_t* status;
+  uint32_t* status;  // start of the workspace
   bool debug;
   bool pdl;
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t s);
+size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P);
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap);
 
 }  // namespace dl

@@ -30,6 +30,7 @@
 //    tokens from expert_ids on the device (no host sync), and CTAs of unused
 //    slots exit at once, so only touched experts are read from HBM.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "dl_device.cuh"
 #include "dl_internal.h"
@@ -45,8 +46,9 @@ struct GemmArgs {
   const uint8_t* w;           // packed weights (expert 0 block for MoE)
   long long w_expert_bytes;   // bytes per expert block (0 for dense)
   const float* w_scale;       // [1] or [E]
-  const uint8_t* xq;          // e4m3 activations [M][K]
-  const float* s_x;           // activation scale
+  const uint8_t* xq;          // e4m3 activations [M][K] (read; or written when x != null)
+  float* s_x;                 // activation scale (read; or written when x != null)
+  const uint16_t* x;          // bf16 activations [M][K]: quantise inside this kernel (dense, small M*K)
   uint32_t* status;
   uint16_t* out;              // bf16 [tokens][ldo]
   const int32_t* expert_ids;  // MoE routing (null for dense)
@@ -62,11 +64,33 @@ struct GemmArgs {
 struct GemmMisc {
   uint32_t tmem_base;
   int abort;
+  float sx;                   // activation scale used by the epilogue
+  float wmax[2];              // per-warp |x| maxima of the fused quantiser
   int n_tok;
   int expert;
   int tokens[kMaxTok];
   uint32_t touched[kMaxExperts / 32];
 };
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float absmax8(uint4 u) {
+  float m = fmaxf(fabsf(bf16_lo(u.x)), fabsf(bf16_hi(u.x)));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(u.y)), fabsf(bf16_hi(u.y))));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(u.z)), fabsf(bf16_hi(u.z))));
+  return fmaxf(m, fmaxf(fabsf(bf16_lo(u.w)), fabsf(bf16_hi(u.w))));
+}
+
+// e4m3 codes of 4 bf16 values (two 32-bit words) scaled by inv: one IEEE
+// rounding for the product, then round-to-nearest-even with saturation.
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float inv) {
+  const __nv_fp8x2_storage_t a = __nv_cvt_float2_to_fp8x2(
+      make_float2(__fmul_rn(bf16_lo(w0), inv), __fmul_rn(bf16_hi(w0), inv)), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t b = __nv_cvt_float2_to_fp8x2(
+      make_float2(__fmul_rn(bf16_lo(w1), inv), __fmul_rn(bf16_hi(w1), inv)), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
+}
 
 template <bool kSwiglu>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid_constant__ GemmArgs a) {
@@ -236,11 +260,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     __syncwarp();
   } else {
     // ---- activation stager: e4m3 rows -> swizzled K-major B operand ----
-    pdl_wait();  // x_q and s_x are written by the preceding quantise kernel
+    pdl_wait();  // x (or x_q and s_x) is written by the preceding kernel
     pdl_trigger();
     const int t = threadIdx.x - 64;
     const int per_row = nkb * 8;  // 16-byte chunks per token row of this K slice
     const int chunks = npad * per_row;
+    if (a.x != nullptr) {
+      // Fused quantiser (A1): amax over the whole [M][K] input, then this CTA's
+      // K slice straight into the B operand.  Same arithmetic as act_quant.cu.
+      const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+      const int nv = (a.M * a.K) >> 3;
+      float m0 = 0.0f, m1 = 0.0f;
+      int i = t;
+      for (; i + 64 < nv; i += 128) {
+        m0 = fmaxf(m0, absmax8(__ldg(xv + i)));
+        m1 = fmaxf(m1, absmax8(__ldg(xv + i + 64)));
+      }
+      if (i < nv) m0 = fmaxf(m0, absmax8(__ldg(xv + i)));
+      float m = fmaxf(m0, m1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) misc->wmax[warp - 2] = m;
+      asm volatile("bar.sync 1, 64;" ::: "memory");  // the two stager warps only
+      const float amax = fmaxf(misc->wmax[0], misc->wmax[1]);
+      const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
+      if (t == 0) misc->sx = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      const bool publish = blockIdx.y == 0 && blockIdx.z == 0;  // one CTA column writes x_q / s_x
+      if (publish && rank == 0 && t == 0) *a.s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      for (int c = t; c < chunks; c += 64) {
+        const int row = c / per_row;
+        const int rem = c - row * per_row;
+        const int kbl = rem >> 3;
+        const int ch = rem & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < n_tok && amax > 0.0f) {
+          const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + kbl) * 128 + ch * 16) >> 3);
+          const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+          v = make_uint4(quant4(u0.x, u0.y, inv), quant4(u0.z, u0.w, inv), quant4(u1.x, u1.y, inv),
+                         quant4(u1.z, u1.w, inv));
+        }
+        if (publish && row < n_tok)
+          *reinterpret_cast<uint4*>(const_cast<uint8_t*>(a.xq) + static_cast<long long>(row) * a.K +
+                                    (kb0 + kbl) * 128 + ch * 16) = v;
+        uint8_t* dst = bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = v;
+      }
+      fence_async_smem();
+      mbar_arrive(xready);
+    } else {
+    if (t == 0) misc->sx = __ldg(a.s_x);
     for (int c = t; c < chunks; c += 64) {
       const int row = c / per_row;
       const int rem = c - row * per_row;
@@ -257,6 +325,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     }
     fence_async_smem();
     mbar_arrive(xready);
+    }
   }
 
   // ---- epilogue: TMEM -> shared partials -> cluster reduction -> bf16 ----------
@@ -283,7 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   tc_fence_before();
   cluster_sync();  // all S partial accumulators are complete and visible
 
-  const float scale = __ldg(a.s_x) * __ldg(a.w_scale + expert);
+  const float scale = misc->sx * __ldg(a.w_scale + expert);
   const int r0 = 128 * rank / S;
   const int rows = 128 * (rank + 1) / S - r0;
   const int items = rows * n_tok;
@@ -293,11 +362,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     const int row = r0 + (it - m * rows);
     const int tok = routed ? misc->tokens[m] : m;
     const uint32_t off_g = part_base + static_cast<uint32_t>((m * 128 + row) * 4);
+    float gv[8], uv[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {  // issue every peer load before the first add
+      if (p < S) {
+        gv[p] = dsmem_ld_f32(dsmem_addr(off_g, p));
+        uv[p] = kSwiglu ? dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p)) : 0.0f;
+      }
+    }
     float g = 0.0f;
     float u = 0.0f;
-    for (int p = 0; p < S; ++p) {
-      g += dsmem_ld_f32(dsmem_addr(off_g, p));
-      if (kSwiglu) u += dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p));
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (p < S) {
+        g += gv[p];
+        u += uv[p];
+      }
     }
     if (kSwiglu) {
       const float yg = g * scale;
@@ -372,6 +452,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   a.w_scale = g.w_scale;
   a.xq = g.xq;
   a.s_x = g.s_x;
+  a.x = g.x;
   a.status = g.status;
   a.out = g.out;
   a.expert_ids = g.expert_ids;

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "dl_fc_qkv_scale": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P, _SZ, _P, _U]),
     "dl_moe_fc13_swiglu_grouped": (_I, [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
     "dl_decode_attn": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
+    "dl_decode_attn_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "dl_read_status": (_I, [_P, _P]),
     "dl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -142,6 +143,10 @@ def dl_decode_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, Lcap, 
     return lib().dl_decode_attn(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(v_cache),
                                 Lcap, _ptr(seq_lens), float(softmax_scale), cluster_size, _ptr(out), _ptr(ws),
                                 _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size) -> int:
+    return int(lib().dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size))
 
 
 def dl_read_status(ws, stream=None) -> int:

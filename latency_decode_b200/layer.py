@@ -47,7 +47,8 @@ class DecodeLayer:
         nq = dl.dl_workspace_bytes(M, self.K)
         self.ws_qkv = torch.zeros(nq, dtype=torch.uint8, device=self.device)
         self.ws_13 = torch.zeros(nq, dtype=torch.uint8, device=self.device)
-        self.ws_attn = torch.zeros(dl.dl_workspace_bytes(0, 0), dtype=torch.uint8, device=self.device)
+        self.Lcap_hint = None
+        self.ws_attn = None
         self.qkv = torch.empty((M, self.N_qkv), dtype=torch.int16, device=self.device)
         self.attn_out = torch.empty((B, T, Hq, d), dtype=torch.int16, device=self.device)
         self.ffn_out = torch.empty((M, self.N2 // 2), dtype=torch.int16, device=self.device)
@@ -61,6 +62,10 @@ class DecodeLayer:
         """x1, x2: bf16 bits [M, K] (int16); k_cache, v_cache: bf16 bits [B, Hkv, Lcap, d];
         seq_lens: int32 [B].  Results land in self.attn_out and self.ffn_out."""
         Lcap = k_cache.shape[2]
+        if self.ws_attn is None or self.Lcap_hint != Lcap:
+            n = dl.dl_decode_attn_workspace_bytes(self.B, self.T, self.Hq, self.Hkv, self.d, Lcap, self.cluster)
+            self.ws_attn = torch.zeros(n, dtype=torch.uint8, device=self.device)
+            self.Lcap_hint = Lcap
         dl.check(dl.dl_fc_qkv_scale(x1, self.M, self.K, self.wp_qkv, self.s_qkv, self.Hq, self.Hkv, self.d,
                                     self.q_scale, self.qkv, self.ws_qkv, stream=stream, flags=flags))
         dl.check(dl.dl_decode_attn(self.qkv, self.N_qkv, self.B, self.T, self.Hq, self.Hkv, self.d, k_cache,
@@ -71,4 +76,5 @@ class DecodeLayer:
 
     def read_status(self, stream=None) -> None:
         for ws in (self.ws_qkv, self.ws_attn, self.ws_13):
-            dl.check(dl.dl_read_status(ws, stream))
+            if ws is not None:
+                dl.check(dl.dl_read_status(ws, stream))

@@ -67,6 +67,13 @@ def test_workspace_bytes():
     assert dl.dl_workspace_bytes(1, 100) == 512
 
 
+def test_attention_workspace_bytes():
+    assert dl.dl_decode_attn_workspace_bytes(1, 1, 40, 8, 128, 4096, 8) > 256  # splits over clusters
+    assert dl.dl_decode_attn_workspace_bytes(16, 4, 40, 8, 128, 16384, 8) == 256  # enough CTAs already
+    assert dl.dl_decode_attn_workspace_bytes(1, 1, 8, 2, 64, 256, 8) == 256  # too short to split
+    assert dl.dl_decode_attn_workspace_bytes(1, 1, 6, 4, 64, 256, 8) == 0  # Hq % Hkv != 0
+
+
 def _fc13(**kw):
     a = dict(x=FAKE, M=1, K=512, w_packed=FAKE, w_scale=FAKE, N2=2048, out=FAKE, ws=FAKE,
              ws_bytes=1 << 20, stream=0, flags=0)

@@ -26,10 +26,14 @@ def lib():
 
 
 def run_attn(q_flat, q_stride, B, T, Hq, Hkv, d, k, v, seq_lens, scale, cluster, flags=dl.DL_FLAG_PDL,
-             expect=dl.DL_OK):
+             expect=dl.DL_OK, splits=0):
     Lcap = k.shape[2]
     out = torch.full((B, T, Hq, d), -1, dtype=torch.int16, device="cuda")
-    ws, n = new_ws(0, 0)
+    n = dl.dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster)
+    if splits:
+        n = max(n, 256 + 4096 + 2 * 65536 + B * Hkv * splits * (Hq // Hkv) * T * d * 4 + 65536)
+        flags |= splits << dl.DL_FLAG_SPLIT_SHIFT
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
     dl.check(dl.dl_decode_attn(dev_u16(q_flat), q_stride, B, T, Hq, Hkv, d, dev_u16(k), dev_u16(v), Lcap,
                                dev_i32(seq_lens), scale, cluster, out, ws, n, flags=flags))
     assert dl.dl_read_status(ws) == expect
@@ -44,10 +48,10 @@ def case(seed, B, T, Hq, Hkv, d, Lcap, seq_lens):
     return q, k, v, np.asarray(seq_lens, dtype=np.int32)
 
 
-def check(seed, B, T, Hq, Hkv, d, Lcap, seq_lens, cluster, scale=None):
+def check(seed, B, T, Hq, Hkv, d, Lcap, seq_lens, cluster, scale=None, splits=0):
     q, k, v, sl = case(seed, B, T, Hq, Hkv, d, Lcap, seq_lens)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    got = run_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, k, v, sl, scale, cluster)
+    got = run_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, k, v, sl, scale, cluster, splits=splits)
     ref = oracle.decode_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, k, v, sl, scale)
     return helpers.check_attn(got, ref, f"B={B} T={T} Hq={Hq} Hkv={Hkv} d={d} L={seq_lens} S={cluster}")
 
@@ -136,6 +140,36 @@ def test_identical_keys_give_mean_of_values():
     for h in range(Hq):
         mean = vf[0, h // 4].mean(axis=0)
         assert helpers.rel_l2(got[0, 0, h], mean) < 5e-3
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 5])
+def test_clusters_per_head_merge_through_workspace(splits):
+    # P clusters per (b, kv head): DSMEM merge inside each, workspace merge across them
+    check(60 + splits, 2, 4, 10, 2, 128, 2000, [2000, 731], 8, splits=splits)
+
+
+@pytest.mark.parametrize("splits", [2, 7])
+def test_clusters_per_head_with_empty_clusters_and_small_d(splits):
+    check(70 + splits, 1, 1, 8, 2, 64, 512, [100], 4, splits=splits)
+
+
+def test_workspace_counters_return_to_zero_and_repeat_calls_agree():
+    B, T, Hq, Hkv, d, L = 1, 1, 40, 8, 128, 4096
+    q, k, v, sl = case(80, B, T, Hq, Hkv, d, L, [L])
+    n = dl.dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, L, 8)
+    assert n > 256  # the batch-1 shape splits each head over several clusters
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    args = (dev_u16(q.ravel()), Hq * d, B, T, Hq, Hkv, d, dev_u16(k), dev_u16(v), L, dev_i32(sl), 0.088, 8)
+    outs = []
+    for _ in range(3):
+        out = torch.empty((B, T, Hq, d), dtype=torch.int16, device="cuda")
+        dl.check(dl.dl_decode_attn(*args, out, ws))
+        assert dl.dl_read_status(ws) == dl.DL_OK
+        outs.append(host_u16(out))
+    assert not ws[256:256 + 4 * B * Hkv].any()  # every per-head counter is back to zero
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
+    ref = oracle.decode_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, k, v, sl, 0.088)
+    helpers.check_attn(outs[0], ref, "repeat calls")
 
 
 def test_bad_seq_len_is_reported_on_device():
