@@ -62,8 +62,19 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
   const int v1 = static_cast<int>(static_cast<long long>(nv) * (r + 1) / C);
   const uint4* xv = reinterpret_cast<const uint4*>(x);
 
+  // eight independent 16-byte loads in flight per thread per round
+  constexpr int kBatch = 8;
   float m = 0.0f;
-  for (int i = v0 + threadIdx.x; i < v1; i += kAqThreads) m = fmaxf(m, absmax8(__ldg(xv + i)));
+  for (int base = v0 + threadIdx.x; base < v1; base += kBatch * kAqThreads) {
+    uint4 u[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + j * kAqThreads;
+      u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) m = fmaxf(m, absmax8(u[j]));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
@@ -83,9 +94,18 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
   uint2* q2 = reinterpret_cast<uint2*>(xq);
   if (amax > 0.0f) {
     const float inv = __fdiv_rn(448.0f, amax);
-    for (int i = v0 + threadIdx.x; i < v1; i += kAqThreads) {
-      const uint4 u = __ldg(xv + i);
-      q2[i] = make_uint2(quant4(u.x, u.y, inv), quant4(u.z, u.w, inv));
+    for (int base = v0 + threadIdx.x; base < v1; base += kBatch * kAqThreads) {
+      uint4 u[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int i = base + j * kAqThreads;
+        u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int i = base + j * kAqThreads;
+        if (i < v1) q2[i] = make_uint2(quant4(u[j].x, u[j].y, inv), quant4(u[j].z, u[j].w, inv));
+      }
     }
   } else {
     for (int i = v0 + threadIdx.x; i < v1; i += kAqThreads) q2[i] = make_uint2(0u, 0u);
@@ -98,7 +118,7 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, uint8_t* xq, float* s_x,
                              cudaStream_t s, bool pdl) {
   const long long n = static_cast<long long>(M) * K;
-  int C = static_cast<int>((n + 65535) / 65536);  // ~64K elements per CTA
+  int C = static_cast<int>((n + 32767) / 32768);  // ~32K elements (64 KB of bf16) per CTA
   if (C < 1) C = 1;
   if (C > 8) C = 8;
   Launch L(dim3(C), dim3(kAqThreads), 0, s, static_cast<unsigned>(C), pdl);

@@ -38,10 +38,12 @@
 
 namespace dl {
 
-constexpr int kAttnKT = 64;           // keys per pipeline stage
-constexpr int kAttnConsumers = 4;     // consumer warps, 16 keys each per stage
-constexpr int kAttnThreads = 32 * (kAttnConsumers + 1);
+// W consumer warps take 16 keys each of a stage of 16*W keys; one more warp
+// is the TMA producer.  W = 4 for up to 16 query rows per kv head (two CTAs
+// per SM), W = 8 for more rows (one CTA per SM, twice the warps to hide the
+// MMA and softmax latency).
 constexpr int kAttnMaxSplits = 16;    // clusters per (b, kv head)
+constexpr int kLazyRescale = 8;       // log2 headroom before the running max is raised
 
 struct AttnArgs {
   const uint16_t* q;
@@ -51,12 +53,12 @@ struct AttnArgs {
   float scale_log2;  // softmax scale * log2(e)
   uint16_t* out;
   uint32_t* status;
-  uint32_t* counters;  // [B*Hkv], P > 1 only
-  float* part_m;       // [B*Hkv][P][R]
-  float* part_l;       // [B*Hkv][P][R]
-  float* part_o;       // [B*Hkv][P][R][D]
+  uint32_t* counters;  // [B*Hkv][S], P > 1 only
+  float* part_ml;      // [B*Hkv][P][S][R][2] per-owner (m, l)
+  float* part_o;       // [B*Hkv][P][R*D/4] float4
   int P;
   int stages;
+  int recv_off;        // byte offset of the DSMEM receive buffer
   int debug;
 };
 
@@ -64,12 +66,15 @@ __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+template <int D, int NT, int W>
+__global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ AttnArgs a) {
+  constexpr int kAttnConsumers = W;
+  constexpr int kAttnThreads = 32 * (W + 1);
+  constexpr int kAttnKT = 16 * W;             // keys per pipeline stage
   constexpr int HALVES = D / 64;              // a swizzled row holds 64 bf16 (128 bytes)
-  constexpr int HALF_BYTES = kAttnKT * 128;   // 64 keys x 128 bytes
+  constexpr int HALF_BYTES = kAttnKT * 128;   // kAttnKT keys x 128 bytes
   constexpr int STAGE_BYTES = 2 * HALVES * HALF_BYTES;
   constexpr int KS = D / 16;                  // MMA k-steps over d, and m-tiles of d
   extern __shared__ uint8_t smem_raw[];
@@ -77,6 +82,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
   uint2* qs = reinterpret_cast<uint2*>(ring + a.stages * STAGE_BYTES);        // [KS][NT][32]
+  uint8_t* recv_base = smem + a.recv_off;                                      // DSMEM receive buffer
   uint64_t* bars = reinterpret_cast<uint64_t*>(qs + KS * NT * 32);
   int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages);
   int* last_word = abort_word + 1;
@@ -255,18 +261,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            const float m_new = fmaxf(m_run[nt][j], mx);
-            const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-            const float alpha = ex2(m_run[nt][j] - m_use);
+            // Lazy rescale: the reference max m_run moves only when this tile's
+            // max exceeds it by more than 2^kLazyRescale, so the O rescale below
+            // is rarely needed; p stays <= 2^kLazyRescale, far from overflow.
+            if (mx > m_run[nt][j] + static_cast<float>(kLazyRescale)) {
+              const float m_new = mx;
+              const float alpha = ex2(m_run[nt][j] - m_new);  // 0 when m_run is -inf
+              l_run[nt][j] *= alpha;
+#pragma unroll
+              for (int mt = 0; mt < KS; ++mt) {
+                o[mt][nt][j] *= alpha;
+                o[mt][nt][2 + j] *= alpha;
+              }
+              m_run[nt][j] = m_new;
+            }
+            const float m_use = (m_run[nt][j] == -INFINITY) ? 0.0f : m_run[nt][j];
             p[j] = ex2(x0 - m_use);
             p[2 + j] = ex2(x1 - m_use);
-            l_run[nt][j] = l_run[nt][j] * alpha + p[j] + p[2 + j];
-            m_run[nt][j] = m_new;
-#pragma unroll
-            for (int mt = 0; mt < KS; ++mt) {
-              o[mt][nt][j] *= alpha;
-              o[mt][nt][2 + j] *= alpha;
-            }
+            l_run[nt][j] += p[j] + p[2 + j];
           }
           // P^T as the B operand [k = key][n = row]: transpose each 8x8 block
           pb[nt][0] = movmatrix_t(pack_bf16x2(p[0], p[1]));
@@ -304,15 +316,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
   }
 
-  __syncthreads();  // the ring is drained: reuse it for the merge buffers
+  __syncthreads();  // the ring is drained: reuse it for the per-warp states
   pdl_wait();
   const int R = a.R;
-  float* wo = reinterpret_cast<float*>(ring);             // [4][R][D] per-warp o
-  float* wm = wo + kAttnConsumers * R * D;                // [4][R]
-  float* wl = wm + kAttnConsumers * R;                    // [4][R]
-  float* cm = wl + kAttnConsumers * R;                    // [R]   CTA state, read by peers
-  float* cl = cm + R;                                     // [R]
-  float* co = cl + R + ((4 - ((2 * R) & 3)) & 3);         // [R][D], 16-byte aligned
+  float* wo = reinterpret_cast<float*>(ring);             // [W][R][D] per-warp o
+  float* wm = wo + kAttnConsumers * R * D;                // [W][R]
+  float* wl = wm + kAttnConsumers * R;                    // [W][R]
   if (warp < kAttnConsumers) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -333,64 +342,76 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
   }
   __syncthreads();
-  // ---- merge the four warp states into this CTA's state ----
-  for (int idx = threadIdx.x; idx < R * D; idx += kAttnThreads) {
-    const int rho = idx / D;
+
+  // ---- merge the four warp states and push the CTA state to the slice owners ----
+  // Outputs are I = R*D/4 float4 items; CTA c of the cluster owns items
+  // [c*Q, (c+1)*Q).  Every CTA stores its state of item i straight into the
+  // receive buffer of the owner of i (remote shared-memory stores, no round
+  // trip), and the (m, l) of each row into every peer; one cluster barrier
+  // later each owner merges the S states of its items locally.
+  const int I = R * (D / 4);
+  const int Q = (I + S - 1) / S;
+  float4* rv_o = reinterpret_cast<float4*>(recv_base);     // [S][Q]
+  float* rv_m = reinterpret_cast<float*>(rv_o + S * Q);   // [S][R]
+  float* rv_l = rv_m + S * R;                             // [S][R]
+  const uint32_t rv_o_l = smem_u32(rv_o), rv_m_l = smem_u32(rv_m), rv_l_l = smem_u32(rv_l);
+  for (int it = threadIdx.x; it < I; it += kAttnThreads) {
+    const int rho = it / (D / 4);
+    const int c4 = it - rho * (D / 4);
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kAttnConsumers; ++w)
       if (wl[w * R + rho] > 0.0f) M = fmaxf(M, wm[w * R + rho]);
-    float acc = 0.0f, lsum = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.0f;
 #pragma unroll
     for (int w = 0; w < kAttnConsumers; ++w) {
       const float lw = wl[w * R + rho];
       if (lw > 0.0f) {
         const float f = ex2(wm[w * R + rho] - M);
-        acc += wo[(w * R + rho) * D + (idx - rho * D)] * f;
-        lsum += lw * f;
-      }
-    }
-    co[idx] = acc;
-    if (idx - rho * D == 0) {
-      cm[rho] = M;
-      cl[rho] = lsum;
-    }
-  }
-  cluster_sync();  // every CTA state of the cluster is visible through DSMEM
-
-  // ---- merge the S CTA states; CTA `rank` handles a 1/S slice of the outputs ----
-  const int items = R * (D / 4);
-  const int i0 = static_cast<int>(static_cast<long long>(items) * rank / S);
-  const int i1 = static_cast<int>(static_cast<long long>(items) * (rank + 1) / S);
-  const uint32_t cm_l = smem_u32(cm), cl_l = smem_u32(cl), co_l = smem_u32(co);
-  const long long head = static_cast<long long>(b) * a.Hkv + hk;
-  for (int it = i0 + threadIdx.x; it < i1; it += kAttnThreads) {
-    const int rho = it / (D / 4);
-    const int c4 = it - rho * (D / 4);
-    float mp[16], lp[16];
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {  // issue every peer load before using them
-      if (p < S) {
-        lp[p] = dsmem_ld_f32(dsmem_addr(cl_l + 4u * rho, p));
-        mp[p] = dsmem_ld_f32(dsmem_addr(cm_l + 4u * rho, p));
-      }
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int p = 0; p < 16; ++p)
-      if (p < S && lp[p] > 0.0f) M = fmaxf(M, mp[p]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.0f;
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-      if (p < S && lp[p] > 0.0f) {
-        const float f = ex2(mp[p] - M);
-        const float4 v = dsmem_ld_f32x4(dsmem_addr(co_l + 4u * (rho * D + c4 * 4), p));
+        const float4 v = *reinterpret_cast<const float4*>(wo + (w * R + rho) * D + c4 * 4);
         acc.x += v.x * f;
         acc.y += v.y * f;
         acc.z += v.z * f;
         acc.w += v.w * f;
-        lsum += lp[p] * f;
+        lsum += lw * f;
+      }
+    }
+    const int owner = it / Q;
+    dsmem_st_f32x4(dsmem_addr(rv_o_l + 16u * (rank * Q + (it - owner * Q)), owner), acc);
+    if (c4 == 0) {
+      for (int p = 0; p < S; ++p) {
+        dsmem_st_f32(dsmem_addr(rv_m_l + 4u * (rank * R + rho), p), M);
+        dsmem_st_f32(dsmem_addr(rv_l_l + 4u * (rank * R + rho), p), lsum);
+      }
+    }
+  }
+  cluster_sync();  // every state of my items has landed in my receive buffer
+
+  // ---- merge the S CTA states of my items ----
+  const long long head = static_cast<long long>(b) * a.Hkv + hk;
+  const long long slot = head * a.P + split;
+  const int my0 = rank * Q;
+  const int cnt = max(0, min(I, my0 + Q) - my0);
+  for (int k = threadIdx.x; k < cnt; k += kAttnThreads) {
+    const int it = my0 + k;
+    const int rho = it / (D / 4);
+    const int c4 = it - rho * (D / 4);
+    float M = -INFINITY;
+    for (int p = 0; p < S; ++p)
+      if (rv_l[p * R + rho] > 0.0f) M = fmaxf(M, rv_m[p * R + rho]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.0f;
+    for (int p = 0; p < S; ++p) {
+      const float lp = rv_l[p * R + rho];
+      if (lp > 0.0f) {
+        const float f = ex2(rv_m[p * R + rho] - M);
+        const float4 v = rv_o[p * Q + k];
+        acc.x += v.x * f;
+        acc.y += v.y * f;
+        acc.z += v.z * f;
+        acc.w += v.w * f;
+        lsum += lp * f;
       }
     }
     if (a.P == 1) {
@@ -403,47 +424,49 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
       *reinterpret_cast<uint2*>(dst) = packed;
     } else {
-      // this cluster's merged state, unnormalised, for the cross-cluster merge
-      const long long slot = head * a.P + split;
-      *reinterpret_cast<float4*>(a.part_o + (slot * R + rho) * D + c4 * 4) = acc;
-      if (c4 == 0) {
-        a.part_m[slot * R + rho] = M;
-        a.part_l[slot * R + rho] = lsum;
+      // this cluster's merged state of my items, unnormalised, for the cross-cluster merge
+      *reinterpret_cast<float4*>(a.part_o + (slot * I + it) * 4) = acc;
+      if (c4 == 0 || k == 0) {
+        float* ml = a.part_ml + ((slot * S + rank) * R + rho) * 2;
+        ml[0] = M;
+        ml[1] = lsum;
       }
     }
   }
   if (a.P > 1) {
+    // The P CTAs that own the same items in the P clusters of this head meet
+    // through the workspace: the last one to arrive merges and stores them.
     __threadfence();
-    cluster_sync();  // every CTA of this cluster has stored and fenced its slice
-    if (rank == 0 && threadIdx.x == 0) {
-      const unsigned prev = atomicAdd(a.counters + head, 1u);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const unsigned prev = atomicAdd(a.counters + head * S + rank, 1u);
       const int last = prev == static_cast<unsigned>(a.P - 1);
       if (last) {
         __threadfence();
-        a.counters[head] = 0u;  // every other cluster of this head has arrived: reset for the next call
+        a.counters[head * S + rank] = 0u;  // all P have arrived: reset for the next call
       }
       *last_word = last;
     }
-    cluster_sync();
-    const int last = static_cast<int>(dsmem_ld_u32(dsmem_addr(smem_u32(last_word), 0)));
-    if (last) {
+    __syncthreads();
+    if (*last_word) {
       __threadfence();
-      for (int it = i0 + threadIdx.x; it < i1; it += kAttnThreads) {
+      for (int k = threadIdx.x; k < cnt; k += kAttnThreads) {
+        const int it = my0 + k;
         const int rho = it / (D / 4);
         const int c4 = it - rho * (D / 4);
         float M = -INFINITY;
         for (int p = 0; p < a.P; ++p) {
-          const long long slot = head * a.P + p;
-          if (__ldcg(a.part_l + slot * R + rho) > 0.0f) M = fmaxf(M, __ldcg(a.part_m + slot * R + rho));
+          const float* ml = a.part_ml + (((head * a.P + p) * S + rank) * R + rho) * 2;
+          if (__ldcg(ml + 1) > 0.0f) M = fmaxf(M, __ldcg(ml));
         }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float lsum = 0.0f;
         for (int p = 0; p < a.P; ++p) {
-          const long long slot = head * a.P + p;
-          const float lq = __ldcg(a.part_l + slot * R + rho);
+          const float* ml = a.part_ml + (((head * a.P + p) * S + rank) * R + rho) * 2;
+          const float lq = __ldcg(ml + 1);
           if (lq > 0.0f) {
-            const float f = ex2(__ldcg(a.part_m + slot * R + rho) - M);
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (slot * R + rho) * D + c4 * 4));
+            const float f = ex2(__ldcg(ml) - M);
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((head * a.P + p) * I + it) * 4));
             acc.x += v.x * f;
             acc.y += v.y * f;
             acc.z += v.z * f;
@@ -462,7 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
   }
-  cluster_sync();  // keep this CTA's state alive until every peer has read it
+  // No trailing cluster barrier: after the one above, no CTA touches another CTA's shared memory.
 }
 
 // ---- host side ----------------------------------------------------------------------
@@ -480,66 +503,138 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-static bool encode_kv_map(CUtensorMap* m, const uint16_t* base, int d, int Lcap, int BH) {
+static bool encode_kv_map(CUtensorMap* m, const uint16_t* base, int d, int Lcap, int BH, int kt) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Lcap), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(Lcap) * d * 2};
-  cuuint32_t box[3] = {64, kAttnKT, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kt), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Workspace of dl_decode_attn with P clusters per (b, kv head): the 256-byte
-// header, then the per-head counters, then the P cluster states.
-size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P) {
+// Workspace of dl_decode_attn with P clusters per (b, kv head) of S CTAs: the
+// 256-byte header, the per-(head, owner) counters, the per-owner (m, l) of each
+// cluster, and the merged item states of each cluster.
+size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P, int S) {
   if (P <= 1) return kWsHeader;
   const size_t heads = static_cast<size_t>(B) * Hkv;
-  const size_t counters = (heads * 4 + 255) / 256 * 256;
-  const size_t ml = (heads * P * R * 4 + 255) / 256 * 256;
-  return kWsHeader + counters + 2 * ml + heads * P * R * d * 4;
+  const size_t counters = (heads * S * 4 + 255) / 256 * 256;
+  const size_t ml = (heads * P * S * R * 2 * 4 + 255) / 256 * 256;
+  return kWsHeader + counters + ml + heads * P * R * d * 4;
 }
 
-int attn_auto_splits(int B, int Hkv, int cluster, int Lcap) {
-  const long long base = static_cast<long long>(B) * Hkv * cluster;
-  const long long target = 2ll * sm_count();  // two CTAs per SM
-  if (base >= target) return 1;
-  long long P = target / base;
-  const long long by_len = Lcap / (static_cast<long long>(cluster) * 2 * kAttnKT);  // >= 2 tiles per CTA
-  if (P > by_len) P = by_len;
+// Shared-memory plan of one attention CTA: two CTAs per SM when a 3-stage
+// ring (6 for d=64) fits, else one CTA per SM with the deepest ring (<= 6
+// stages) that fits.  The per-warp merge buffers reuse the drained ring.
+struct AttnPlan {
+  int stages, smem, recv_off;
+};
+
+template <int D, int NT, int W>
+static AttnPlan attn_plan(int R, int S) {
+  constexpr int STAGE_BYTES = 2 * (D / 64) * (16 * W) * 128;
+  const int merge_bytes = (W * R * D + 2 * W * R) * 4;
+  const int I = R * (D / 4);
+  const int Q = (I + S - 1) / S;
+  const int recv_bytes = S * Q * 16 + 2 * S * R * 4;
+  const int qs_bytes = (D / 16) * NT * 32 * 8;
+  auto smem_for = [&](int st) { return 1024 + st * STAGE_BYTES + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16; };
+  int stages = W == 4 ? (D == 128 ? 3 : 6) : (D == 128 ? 3 : 6);
+  if (W == 8 || 2 * (smem_for(stages) + 1024) > 233472) {
+    stages = 6;
+    while (stages > 2 && smem_for(stages) > 232448) --stages;
+  }
+  while (stages * STAGE_BYTES < merge_bytes) ++stages;
+  AttnPlan pl;
+  pl.stages = stages;
+  pl.smem = smem_for(stages);
+  pl.recv_off = ((stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
+  return pl;
+}
+
+template <int D, int NT, int W>
+static cudaError_t attn_configure(const AttnPlan& pl, int S) {
+  auto kern = decode_attn_kernel<D, NT, W>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+  if (e == cudaSuccess && S > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+// Clusters of S CTAs of this kernel that can be resident on the GPU at once.
+template <int D, int NT, int W>
+static int attn_max_clusters_t(int R, int S) {
+  const AttnPlan pl = attn_plan<D, NT, W>(R, S);
+  const int per_sm = 233472 / (pl.smem + 1024) >= 2 ? 2 : 1;
+  int fallback = (sm_count() * per_sm) / S;
+  if (attn_configure<D, NT, W>(pl, S) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fallback;
+  }
+  Launch L(dim3(S, 1, 1), dim3(32 * (W + 1)), static_cast<size_t>(pl.smem), nullptr, static_cast<unsigned>(S), false);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, NT, W>, &L.cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    return fallback;
+  }
+  return n;
+}
+
+static int attn_max_clusters(int d, int R, int S) {
+  const int NT = (R + 7) / 8;
+  if (d == 128) {
+    switch (NT) {
+      case 1: return attn_max_clusters_t<128, 1, 4>(R, S);
+      case 2: return attn_max_clusters_t<128, 2, 4>(R, S);
+      case 3: return attn_max_clusters_t<128, 3, 8>(R, S);
+      default: return attn_max_clusters_t<128, 4, 8>(R, S);
+    }
+  }
+  switch (NT) {
+    case 1: return attn_max_clusters_t<64, 1, 4>(R, S);
+    case 2: return attn_max_clusters_t<64, 2, 4>(R, S);
+    case 3: return attn_max_clusters_t<64, 3, 8>(R, S);
+    default: return attn_max_clusters_t<64, 4, 8>(R, S);
+  }
+}
+
+// Clusters per (b, kv head).  Splitting a head over P clusters costs a merge
+// through the workspace (~2-3 us), so it is used only when each CTA would
+// otherwise stream long chunks (>= 2048 keys), with >= 1024 keys per CTA
+// left, and never beyond the clusters that can be resident at once.
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R) {
+  const long long keys_per_cta = Lcap / cluster;
+  if (keys_per_cta < 2048) return 1;
+  const long long heads = static_cast<long long>(B) * Hkv;
+  const long long resident = attn_max_clusters(d, R, cluster);
+  long long P = resident / heads;
+  if (P > keys_per_cta / 1024) P = keys_per_cta / 1024;
   if (P > kAttnMaxSplits) P = kAttnMaxSplits;
   return P < 1 ? 1 : static_cast<int>(P);
 }
 
-template <int D, int NT>
+template <int D, int NT, int W>
 static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                                  const AttnLaunch& p, cudaStream_t s) {
-  constexpr int STAGE_BYTES = 2 * (D / 64) * kAttnKT * 128;
-  const int R = a.R;
-  const int merge_bytes = (kAttnConsumers * R * D + 2 * kAttnConsumers * R + 2 * R + 4 + R * D) * 4;
-  int stages = D == 128 ? 3 : 6;  // ~100 KB of ring: two CTAs per SM
-  while (stages * STAGE_BYTES < merge_bytes) ++stages;
+  const AttnPlan pl = attn_plan<D, NT, W>(a.R, p.cluster);
   AttnArgs args = a;
-  args.stages = stages;
-  const int qs_bytes = (D / 16) * NT * 32 * 8;
-  const int smem = 1024 + stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16;
-  auto kern = decode_attn_kernel<D, NT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  args.stages = pl.stages;
+  args.recv_off = pl.recv_off;
+  cudaError_t e = attn_configure<D, NT, W>(pl, p.cluster);
   if (e != cudaSuccess) return e;
-  if (p.cluster > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  Launch L(dim3(p.cluster, p.Hkv, p.B * a.P), dim3(kAttnThreads), static_cast<size_t>(smem), s,
+  Launch L(dim3(p.cluster, p.Hkv, p.B * a.P), dim3(32 * (W + 1)), static_cast<size_t>(pl.smem), s,
            static_cast<unsigned>(p.cluster), p.pdl);
-  return cudaLaunchKernelEx(&L.cfg, kern, tk, tv, args);
+  return cudaLaunchKernelEx(&L.cfg, decode_attn_kernel<D, NT, W>, tk, tv, args);
 }
 
 cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
+  const int R_ = (p.Hq / p.Hkv) * p.T;
+  const int kt = 16 * ((R_ + 7) / 8 >= 3 ? 8 : 4);  // keys per stage of the chosen variant
   CUtensorMap tk, tv;
-  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv) || !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv))
+  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt) ||
+      !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = p.q;
@@ -558,36 +653,35 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   a.stages = 3;
   a.debug = p.debug ? 1 : 0;
   // clusters per (b, kv head): forced, else automatic; then as many as the workspace holds
-  int P = p.splits > 0 ? p.splits : attn_auto_splits(p.B, p.Hkv, p.cluster, p.Lcap);
-  while (P > 1 && attn_ws_bytes(p.B, p.Hkv, a.R, p.d, P) > p.ws_bytes) --P;
+  int P = p.splits > 0 ? p.splits : attn_auto_splits(p.B, p.Hkv, p.cluster, p.Lcap, p.d, a.R);
+  while (P > 1 && attn_ws_bytes(p.B, p.Hkv, a.R, p.d, P, p.cluster) > p.ws_bytes) --P;
   if (static_cast<long long>(p.B) * P > 65535) P = 1;
   a.P = P;
   a.counters = nullptr;
-  a.part_m = a.part_l = a.part_o = nullptr;
+  a.part_ml = a.part_o = nullptr;
   if (P > 1) {
     const size_t heads = static_cast<size_t>(p.B) * p.Hkv;
     uint8_t* base = reinterpret_cast<uint8_t*>(p.status) + kWsHeader;
     a.counters = reinterpret_cast<uint32_t*>(base);
-    base += (heads * 4 + 255) / 256 * 256;
-    const size_t ml = (heads * P * a.R * 4 + 255) / 256 * 256;
-    a.part_m = reinterpret_cast<float*>(base);
-    a.part_l = reinterpret_cast<float*>(base + ml);
-    a.part_o = reinterpret_cast<float*>(base + 2 * ml);
+    base += (heads * p.cluster * 4 + 255) / 256 * 256;
+    a.part_ml = reinterpret_cast<float*>(base);
+    base += (heads * P * p.cluster * a.R * 2 * 4 + 255) / 256 * 256;
+    a.part_o = reinterpret_cast<float*>(base);
   }
   const int NT = (a.R + 7) / 8;
   if (p.d == 128) {
     switch (NT) {
-      case 1: return launch_attn_t<128, 1>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<128, 2>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<128, 3>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<128, 4>(tk, tv, a, p, s);
+      case 1: return launch_attn_t<128, 1, 4>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<128, 2, 4>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<128, 3, 8>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<128, 4, 8>(tk, tv, a, p, s);
     }
   } else if (p.d == 64) {
     switch (NT) {
-      case 1: return launch_attn_t<64, 1>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<64, 2>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<64, 3>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<64, 4>(tk, tv, a, p, s);
+      case 1: return launch_attn_t<64, 1, 4>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<64, 2, 4>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<64, 3, 8>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<64, 4, 8>(tk, tv, a, p, s);
     }
   }
   return cudaErrorInvalidValue;

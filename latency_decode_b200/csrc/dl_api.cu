@@ -61,8 +61,9 @@ size_t dl_workspace_bytes(int M, int K) {
 
 size_t dl_decode_attn_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Lcap, int cluster_size) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || d < 1 || Lcap < 1 || cluster_size < 1 || Hq % Hkv != 0) return 0;
-  const int P = dl::attn_auto_splits(B, Hkv, cluster_size, Lcap);
-  return dl::attn_ws_bytes(B, Hkv, (Hq / Hkv) * T, d, P);
+  if (d != 64 && d != 128) return 0;
+  const int P = dl::attn_auto_splits(B, Hkv, cluster_size, Lcap, d, (Hq / Hkv) * T);
+  return dl::attn_ws_bytes(B, Hkv, (Hq / Hkv) * T, d, P, cluster_size);
 }
 
 dl_status dl_pack_fp8_weight(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,

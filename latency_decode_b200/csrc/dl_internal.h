@@ -90,7 +90,7 @@ struct AttnLaunch {
   bool pdl;
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t s);
-size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P);
-int attn_auto_splits(int B, int Hkv, int cluster, int Lcap);
+size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P, int S);
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R);
 
 }  // namespace dl

@@ -41,6 +41,7 @@ constexpr int kGemmThreads = 128;
 constexpr int kSubBytes = 16384;  // one packed block: 128 rows x 128 K-bytes
 constexpr int kMaxTok = 64;
 constexpr int kMaxExperts = 1024;
+constexpr int kBStages = 4;       // B ring depth when the activations stream in with the weights
 
 struct GemmArgs {
   const uint8_t* w;           // packed weights (expert 0 block for MoE)
@@ -58,6 +59,7 @@ struct GemmArgs {
   int stages;
   int bsm_bytes;
   int tmem_cols;
+  int recv_bytes;             // > 0: split-K partials are pushed into a dedicated receive buffer
   int debug;
 };
 
@@ -101,11 +103,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   uint8_t* ring = smem;
   uint8_t* bsm = ring + a.stages * kSubBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(bsm + a.bsm_bytes);
-  GemmMisc* misc = reinterpret_cast<GemmMisc*>(bars + 2 * a.stages + 2);
+  GemmMisc* misc = reinterpret_cast<GemmMisc*>(bars + 2 * a.stages + 2 + 2 * kBStages);
+  float* recv = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(misc) + ((sizeof(GemmMisc) + 15) & ~15));
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8u * a.stages;
   const uint32_t xready = empty0 + 8u * a.stages;
   const uint32_t done = xready + 8u;
+  const uint32_t bfull0 = done + 8u;                 // B ring (streamed activations)
+  const uint32_t bempty0 = bfull0 + 8u * kBStages;
+  // Fused quantiser: the whole B slice is written once (xready).  Otherwise the
+  // e4m3 activations stream through a kBStages ring beside the weight ring.
+  const bool stream_b = a.x == nullptr;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -186,6 +194,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     }
     mbar_init(xready, 64);
     mbar_init(done, 1);
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(bfull0 + 8u * s, 64);
+      mbar_init(bempty0 + 8u * s, 1);
+    }
     misc->abort = 0;
     fence_mbar_init();
   }
@@ -228,23 +240,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     // ---- MMA issuer ----
     if (lane == 0) {
       int n_mma = 0;
-      if (!mbar_wait(xready, 0, budget, abort_flag)) {
+      if (!stream_b && !mbar_wait(xready, 0, budget, abort_flag)) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
       } else {
         const uint32_t idesc = e4m3_idesc(128, npad);
         for (int i = 0; i < nsub; ++i) {
           const int s = i % a.stages;
+          const int kbl = i / SUBS;
+          const int which = i % SUBS;
+          const int bslot = kbl % kBStages;
+          if (stream_b && which == 0 &&
+              !mbar_wait(bfull0 + 8u * bslot, static_cast<uint32_t>(kbl / kBStages) & 1u, budget, abort_flag)) {
+            set_status(a.status, kStatusTimeout);
+            *abort_flag = 1;
+            break;
+          }
           if (!mbar_wait(full0 + 8u * s, static_cast<uint32_t>(i / a.stages) & 1u, budget, abort_flag)) {
             set_status(a.status, kStatusTimeout);
             *abort_flag = 1;
             break;
           }
           tc_fence_after();
-          const int kbl = i / SUBS;
-          const int which = i % SUBS;
           const uint64_t adesc = sw128_kmajor_desc(smem_u32(ring + s * kSubBytes));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(bsm + kbl * npad * 128));
+          const uint64_t bdesc =
+              sw128_kmajor_desc(smem_u32(bsm + (stream_b ? bslot : kbl) * npad * 128));
 #pragma unroll
           for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte swizzle row
             tc_mma_e4m3(tmem + static_cast<uint32_t>(which * npad), adesc + 2u * k, bdesc + 2u * k, idesc,
@@ -252,6 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
           }
           ++n_mma;
           tc_commit(empty0 + 8u * s);  // stage free once these MMAs have read it
+          if (stream_b && which == SUBS - 1) tc_commit(bempty0 + 8u * bslot);  // B slot free too
         }
       }
       if (n_mma > 0) tc_commit(done);
@@ -270,6 +291,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       // K slice straight into the B operand.  Same arithmetic as act_quant.cu.
       const uint4* xv = reinterpret_cast<const uint4*>(a.x);
       const int nv = (a.M * a.K) >> 3;
+      // This thread's first kKeep chunks of the CTA's K slice are loaded into
+      // registers in the same batch as the amax loads, so quantising them
+      // needs no second trip to memory.
+      constexpr int kKeep = 4;
+      uint4 keep[2 * kKeep];
+#pragma unroll
+      for (int j = 0; j < kKeep; ++j) {
+        keep[2 * j] = make_uint4(0u, 0u, 0u, 0u);
+        keep[2 * j + 1] = keep[2 * j];
+        const int c = t + 64 * j;
+        const int row = c / per_row;
+        if (c < chunks && row < n_tok) {
+          const int rem = c - row * per_row;
+          const uint4* src =
+              xv + ((static_cast<long long>(row) * a.K + (kb0 + (rem >> 3)) * 128 + (rem & 7) * 16) >> 3);
+          keep[2 * j] = __ldg(src);
+          keep[2 * j + 1] = __ldg(src + 1);
+        }
+      }
       float m0 = 0.0f, m1 = 0.0f;
       int i = t;
       for (; i + 64 < nv; i += 128) {
@@ -287,15 +327,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       if (t == 0) misc->sx = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
       const bool publish = blockIdx.y == 0 && blockIdx.z == 0;  // one CTA column writes x_q / s_x
       if (publish && rank == 0 && t == 0) *a.s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      for (int c = t; c < chunks; c += 64) {
+      for (int c = t, j = 0; c < chunks; c += 64, ++j) {
         const int row = c / per_row;
         const int rem = c - row * per_row;
         const int kbl = rem >> 3;
         const int ch = rem & 7;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (row < n_tok && amax > 0.0f) {
-          const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + kbl) * 128 + ch * 16) >> 3);
-          const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+          uint4 u0, u1;
+          if (j < kKeep) {
+#pragma unroll
+            for (int q = 0; q < kKeep; ++q)
+              if (q == j) {
+                u0 = keep[2 * q];
+                u1 = keep[2 * q + 1];
+              }
+          } else {
+            const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + kbl) * 128 + ch * 16) >> 3);
+            u0 = __ldg(src);
+            u1 = __ldg(src + 1);
+          }
           v = make_uint4(quant4(u0.x, u0.y, inv), quant4(u0.z, u0.w, inv), quant4(u1.x, u1.y, inv),
                          quant4(u1.z, u1.w, inv));
         }
@@ -309,22 +360,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       mbar_arrive(xready);
     } else {
     if (t == 0) misc->sx = __ldg(a.s_x);
-    for (int c = t; c < chunks; c += 64) {
-      const int row = c / per_row;
-      const int rem = c - row * per_row;
-      const int kbl = rem >> 3;
-      const int ch = rem & 7;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < n_tok) {
-        const int tok = routed ? misc->tokens[row] : row;
-        v = *reinterpret_cast<const uint4*>(a.xq + static_cast<long long>(tok) * a.K + (kb0 + kbl) * 128 +
-                                            ch * 16);
+    // Stream the e4m3 activations of each k-block into the B ring, one slot
+    // ahead of the MMAs that read it; every 16-byte chunk is an independent
+    // async copy, so a whole k-block is in flight at once.
+    for (int kbl = 0; kbl < nkb; ++kbl) {
+      const int bslot = kbl % kBStages;
+      if (kbl >= kBStages &&
+          !mbar_wait(bempty0 + 8u * bslot, static_cast<uint32_t>((kbl / kBStages) - 1) & 1u, budget, abort_flag)) {
+        set_status(a.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
       }
-      uint8_t* dst = bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = v;
+      uint8_t* blk = bsm + bslot * npad * 128;
+      for (int c = t; c < npad * 8; c += 64) {
+        const int row = c >> 3;
+        const int ch = c & 7;
+        uint8_t* dst = blk + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
+        if (row < n_tok) {
+          const int tok = routed ? misc->tokens[row] : row;
+          cp_async_16(smem_u32(dst), a.xq + static_cast<long long>(tok) * a.K + (kb0 + kbl) * 128 + ch * 16);
+        } else {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      cp_async_wait_all();
+      fence_async_smem();
+      mbar_arrive(bfull0 + 8u * bslot);
     }
-    fence_async_smem();
-    mbar_arrive(xready);
     }
   }
 
@@ -333,7 +395,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   tc_fence_after();
   pdl_wait();
   fence_async_smem();
-  float* part = reinterpret_cast<float*>(ring);  // [SUBS*npad][128], reuses the drained ring
+  const float scale_w = __ldg(a.w_scale + expert);
+  if (a.recv_bytes > 0) {
+    // Push: each thread owns one accumulator row (its TMEM lane) and stores it
+    // straight into the receive buffer of the CTA that owns that output row;
+    // one cluster barrier later every owner holds all S partials locally.
+    const int Qr = (128 + S - 1) / S;
+    const int row = warp * 32 + lane;
+    const int owner = row / Qr;
+    const int k = row - owner * Qr;
+    const uint32_t dst = dsmem_addr(smem_u32(recv), static_cast<uint32_t>(owner));
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int c0 = 0; c0 < SUBS * npad; c0 += 8) {
+      uint32_t r[8];
+      tmem_ld_x8(lane_base + static_cast<uint32_t>(c0), r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int col = c0 + j;
+        const int which = col / npad;
+        const int m = col - which * npad;
+        if (m < n_tok)
+          dsmem_st_f32(dst + static_cast<uint32_t>((((rank * SUBS + which) * npad + m) * Qr + k) * 4),
+                       __uint_as_float(r[j]));
+      }
+    }
+    tc_fence_before();
+    cluster_sync();  // every partial of my rows has landed in my receive buffer
+    const float scale = misc->sx * scale_w;
+    const int rows = min(Qr, 128 - rank * Qr);
+    const int items = rows > 0 ? rows * n_tok : 0;
+    for (int it = threadIdx.x; it < items; it += kGemmThreads) {
+      const int m = it / rows;
+      const int kk = it - m * rows;
+      const int orow = rank * Qr + kk;
+      const int tok = routed ? misc->tokens[m] : m;
+      float g = 0.0f;
+      float u = 0.0f;
+      for (int p = 0; p < S; ++p) {
+        g += recv[((p * SUBS + 0) * npad + m) * Qr + kk];
+        if (kSwiglu) u += recv[((p * SUBS + 1) * npad + m) * Qr + kk];
+      }
+      if (kSwiglu) {
+        const float yg = g * scale;
+        const float yu = u * scale;
+        const float o = yg / (1.0f + expf(-yg)) * yu;
+        const __nv_bfloat16 bv = __float2bfloat16_rn(o);
+        a.out[static_cast<long long>(tok) * a.ldo + tile * 128 + orow] = *reinterpret_cast<const uint16_t*>(&bv);
+      } else {
+        const int col = tile * 128 + orow;
+        float y = g * scale;
+        if (col < a.q_cols) y *= a.q_scale;
+        const __nv_bfloat16 bv = __float2bfloat16_rn(y);
+        a.out[static_cast<long long>(tok) * a.ldo + col] = *reinterpret_cast<const uint16_t*>(&bv);
+      }
+    }
+    if (warp == 2) {
+      tc_fence_after();
+      tmem_dealloc(tmem, static_cast<uint32_t>(a.tmem_cols));
+    }
+    return;
+  }
+  // Pull (large M): partials parked in the drained ring, summed through DSMEM loads.
+  float* part = reinterpret_cast<float*>(ring);  // [SUBS*npad][128]
   {
     const int row = warp * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
@@ -352,7 +476,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   tc_fence_before();
   cluster_sync();  // all S partial accumulators are complete and visible
 
-  const float scale = misc->sx * __ldg(a.w_scale + expert);
+  const float scale = misc->sx * scale_w;
   const int r0 = 128 * rank / S;
   const int rows = 128 * (rank + 1) / S - r0;
   const int items = rows * n_tok;
@@ -415,27 +539,35 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   const int b_per_kb = npad_max * 128;
   const int sms = sm_count();
 
-  // split-K: enough CTAs for ~2 per SM, at least enough that each CTA's slice of
-  // the activations fits the B buffer, at most 8 (portable cluster) and KB.
+  // split-K: about 1.6 CTAs per SM (measured best at batch 1-4), at least
+  // enough that each CTA's slice of the activations fits the B buffer, at most
+  // 8 (portable cluster) and KB.
+  const bool stream_b = g.x == nullptr;
   int S;
   if (g.split > 0) {
     S = g.split;
   } else {
-    S = (2 * sms) / (n_tiles * g.slots);
-    const int s_fit = (KB * b_per_kb + 45055) / 45056;  // keep B <= 44 KB when possible
-    if (s_fit <= 8 && S < s_fit) S = s_fit;
+    S = (16 * sms / (n_tiles * g.slots) + 5) / 10;
+    const int s_fit = (KB * b_per_kb + 45055) / 45056;  // keep a preloaded B <= 44 KB when possible
+    if (!stream_b && s_fit <= 8 && S < s_fit) S = s_fit;
   }
-  const int s_min = (KB * b_per_kb + 65535) / 65536;  // hard cap: B <= 64 KB
+  const int s_min = stream_b ? 1 : (KB * b_per_kb + 65535) / 65536;  // hard cap: preloaded B <= 64 KB
   if (S < s_min) S = s_min;
   if (S < 1) S = 1;
   if (S > 8) S = 8;
   if (S > KB) S = KB;
   if (S < s_min) return cudaErrorInvalidValue;
   const int nkb_max = (KB + S - 1) / S;
-  const int bsm_bytes = nkb_max * b_per_kb;
+  const int bsm_bytes = stream_b ? kBStages * b_per_kb : nkb_max * b_per_kb;
   const int part_bytes = SUBS * npad_max * 128 * 4;
-  const int misc_bytes = static_cast<int>(sizeof(GemmMisc));
-  auto smem_for = [&](int st) { return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 2) * 8 + misc_bytes; };
+  // split-K partials are pushed into a dedicated receive buffer when it is small
+  const int Qr = (128 + S - 1) / S;
+  int recv_bytes = S * Qr * SUBS * npad_max * 4;
+  if (recv_bytes > 20 * 1024 || S == 1) recv_bytes = 0;
+  const int misc_bytes = static_cast<int>((sizeof(GemmMisc) + 15) & ~static_cast<size_t>(15)) + recv_bytes;
+  auto smem_for = [&](int st) {
+    return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 2 + 2 * kBStages) * 8 + misc_bytes;
+  };
   int stages = 6;
   if (2 * (smem_for(6) + 1024) > 233472) stages = 4;
   if (2 * (smem_for(4) + 1024) > 233472) stages = 6;  // one CTA per SM: keep the deep ring
@@ -466,6 +598,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   a.stages = stages;
   a.bsm_bytes = bsm_bytes;
   a.tmem_cols = tmem_cols;
+  a.recv_bytes = recv_bytes;
   a.debug = g.debug ? 1 : 0;
 
   Launch L(dim3(S, n_tiles, g.slots), dim3(kGemmThreads), static_cast<size_t>(smem), s,

@@ -68,7 +68,8 @@ def test_workspace_bytes():
 
 
 def test_attention_workspace_bytes():
-    assert dl.dl_decode_attn_workspace_bytes(1, 1, 40, 8, 128, 4096, 8) > 256  # splits over clusters
+    assert dl.dl_decode_attn_workspace_bytes(1, 4, 40, 8, 128, 32768, 8) > 256  # long: splits over clusters
+    assert dl.dl_decode_attn_workspace_bytes(1, 1, 40, 8, 128, 4096, 8) == 256  # batch-1 layer: one cluster
     assert dl.dl_decode_attn_workspace_bytes(16, 4, 40, 8, 128, 16384, 8) == 256  # enough CTAs already
     assert dl.dl_decode_attn_workspace_bytes(1, 1, 8, 2, 64, 256, 8) == 256  # too short to split
     assert dl.dl_decode_attn_workspace_bytes(1, 1, 6, 4, 64, 256, 8) == 0  # Hq % Hkv != 0

@@ -154,19 +154,19 @@ def test_clusters_per_head_with_empty_clusters_and_small_d(splits):
 
 
 def test_workspace_counters_return_to_zero_and_repeat_calls_agree():
-    B, T, Hq, Hkv, d, L = 1, 1, 40, 8, 128, 4096
+    B, T, Hq, Hkv, d, L = 1, 4, 40, 8, 128, 8192
     q, k, v, sl = case(80, B, T, Hq, Hkv, d, L, [L])
-    n = dl.dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, L, 8)
-    assert n > 256  # the batch-1 shape splits each head over several clusters
+    n = dl.dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, L, 4)
+    assert n > 256  # long sequences split each head over several clusters
     ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
-    args = (dev_u16(q.ravel()), Hq * d, B, T, Hq, Hkv, d, dev_u16(k), dev_u16(v), L, dev_i32(sl), 0.088, 8)
+    args = (dev_u16(q.ravel()), Hq * d, B, T, Hq, Hkv, d, dev_u16(k), dev_u16(v), L, dev_i32(sl), 0.088, 4)
     outs = []
     for _ in range(3):
         out = torch.empty((B, T, Hq, d), dtype=torch.int16, device="cuda")
         dl.check(dl.dl_decode_attn(*args, out, ws))
         assert dl.dl_read_status(ws) == dl.DL_OK
         outs.append(host_u16(out))
-    assert not ws[256:256 + 4 * B * Hkv].any()  # every per-head counter is back to zero
+    assert not ws[256:256 + 4 * B * Hkv * 4].any()  # every per-(head, owner) counter is back to zero
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
     ref = oracle.decode_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, k, v, sl, 0.088)
     helpers.check_attn(outs[0], ref, "repeat calls")
