@@ -39,9 +39,9 @@
 namespace dl {
 
 // W consumer warps take 16 keys each of a stage of 16*W keys; one more warp
-// is the TMA producer.  W = 4 for up to 16 query rows per kv head (two CTAs
-// per SM), W = 8 for more rows (one CTA per SM, twice the warps to hide the
-// MMA and softmax latency).
+// is the TMA producer.  W = 8 (one CTA per SM, enough warps to hide the MMA and
+// softmax latency) for clusters of up to 8 CTAs; W = 4 (two CTAs per SM where
+// they fit) for 16-CTA clusters, which pack onto the GPCs only that way.
 constexpr int kAttnMaxSplits = 16;    // clusters per (b, kv head)
 constexpr int kLazyRescale = 8;       // log2 headroom before the running max is raised
 
@@ -582,22 +582,29 @@ static int attn_max_clusters_t(int R, int S) {
   return n;
 }
 
-static int attn_max_clusters(int d, int R, int S) {
+static int attn_warps(int S) { return S >= 16 ? 4 : 8; }
+
+template <int W>
+static int attn_max_clusters_w(int d, int R, int S) {
   const int NT = (R + 7) / 8;
   if (d == 128) {
     switch (NT) {
-      case 1: return attn_max_clusters_t<128, 1, 4>(R, S);
-      case 2: return attn_max_clusters_t<128, 2, 4>(R, S);
-      case 3: return attn_max_clusters_t<128, 3, 8>(R, S);
-      default: return attn_max_clusters_t<128, 4, 8>(R, S);
+      case 1: return attn_max_clusters_t<128, 1, W>(R, S);
+      case 2: return attn_max_clusters_t<128, 2, W>(R, S);
+      case 3: return attn_max_clusters_t<128, 3, W>(R, S);
+      default: return attn_max_clusters_t<128, 4, W>(R, S);
     }
   }
   switch (NT) {
-    case 1: return attn_max_clusters_t<64, 1, 4>(R, S);
-    case 2: return attn_max_clusters_t<64, 2, 4>(R, S);
-    case 3: return attn_max_clusters_t<64, 3, 8>(R, S);
-    default: return attn_max_clusters_t<64, 4, 8>(R, S);
+    case 1: return attn_max_clusters_t<64, 1, W>(R, S);
+    case 2: return attn_max_clusters_t<64, 2, W>(R, S);
+    case 3: return attn_max_clusters_t<64, 3, W>(R, S);
+    default: return attn_max_clusters_t<64, 4, W>(R, S);
   }
+}
+
+static int attn_max_clusters(int d, int R, int S) {
+  return attn_warps(S) == 8 ? attn_max_clusters_w<8>(d, R, S) : attn_max_clusters_w<4>(d, R, S);
 }
 
 // Clusters per (b, kv head).  Splitting a head over P clusters costs a merge
@@ -629,9 +636,30 @@ static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, c
   return cudaLaunchKernelEx(&L.cfg, decode_attn_kernel<D, NT, W>, tk, tv, args);
 }
 
+template <int W>
+static cudaError_t launch_attn_w(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
+                                 const AttnLaunch& p, cudaStream_t s, int NT) {
+  if (p.d == 128) {
+    switch (NT) {
+      case 1: return launch_attn_t<128, 1, W>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<128, 2, W>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<128, 3, W>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<128, 4, W>(tk, tv, a, p, s);
+    }
+  } else if (p.d == 64) {
+    switch (NT) {
+      case 1: return launch_attn_t<64, 1, W>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<64, 2, W>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<64, 3, W>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<64, 4, W>(tk, tv, a, p, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
-  const int R_ = (p.Hq / p.Hkv) * p.T;
-  const int kt = 16 * ((R_ + 7) / 8 >= 3 ? 8 : 4);  // keys per stage of the chosen variant
+  const int W = attn_warps(p.cluster);
+  const int kt = 16 * W;  // keys per stage of the chosen variant
   CUtensorMap tk, tv;
   if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt) ||
       !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt))
@@ -669,22 +697,8 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
     a.part_o = reinterpret_cast<float*>(base);
   }
   const int NT = (a.R + 7) / 8;
-  if (p.d == 128) {
-    switch (NT) {
-      case 1: return launch_attn_t<128, 1, 4>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<128, 2, 4>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<128, 3, 8>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<128, 4, 8>(tk, tv, a, p, s);
-    }
-  } else if (p.d == 64) {
-    switch (NT) {
-      case 1: return launch_attn_t<64, 1, 4>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<64, 2, 4>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<64, 3, 8>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<64, 4, 8>(tk, tv, a, p, s);
-    }
-  }
-  return cudaErrorInvalidValue;
+  if (W == 8) return launch_attn_w<8>(tk, tv, a, p, s, NT);
+  return launch_attn_w<4>(tk, tv, a, p, s, NT);
 }
 
 }  // namespace dl

@@ -568,9 +568,10 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   auto smem_for = [&](int st) {
     return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 2 + 2 * kBStages) * 8 + misc_bytes;
   };
+  // the deepest ring (<= 6 stages) that keeps two CTAs per SM, else 6 stages at one CTA per SM
   int stages = 6;
-  if (2 * (smem_for(6) + 1024) > 233472) stages = 4;
-  if (2 * (smem_for(4) + 1024) > 233472) stages = 6;  // one CTA per SM: keep the deep ring
+  while (stages > 3 && 2 * (smem_for(stages) + 1024) > 233472) --stages;
+  if (2 * (smem_for(stages) + 1024) > 233472) stages = 6;
   while (stages * kSubBytes < part_bytes) ++stages;
   int smem = smem_for(stages);
   if (smem > 232448) return cudaErrorInvalidValue;
