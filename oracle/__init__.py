@@ -58,6 +58,10 @@ def _load():
             "oracle_fc_qkv_scale_q": (None, [_P, _F, _P, _F, _I, _I, _I, _I, _I, _F, _P]),
             "oracle_fc_qkv_scale": (None, [_P, _I, _I, _P, _F, _I, _I, _I, _F, _P]),
             "oracle_moe_fc13_swiglu": (None, [_P, _I, _I, _P, _I, _P, _P, _I, _P]),
+            "oracle_linear": (None, [_P, _I, _I, _P, _F, _I, _P]),
+            "oracle_moe_linear": (None, [_P, _I, _I, _P, _I, _P, _P, _I, _P]),
+            "oracle_add_rmsnorm": (None, [_P, _P, _P, _I, _I, _F, _P, _P]),
+            "oracle_quant_f32": (None, [_P, _LL, _P, _P]),
             "oracle_decode_attn": (None, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _P]),
             "oracle_attn_partial": (None, [_P, _LL, _I, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I,
                                            _F, _I, _I, _P, _P, _P]),
@@ -201,6 +205,68 @@ def moe_fc13_swiglu(x_bf16, ids, w, s_w) -> np.ndarray:
     out = np.zeros((T, N2 // 2), dtype=np.float64)
     lib.oracle_moe_fc13_swiglu(_ptr(x), T, K, _ptr(ids), E, _ptr(w), _ptr(s_w), N2, _ptr(out))
     return out
+
+
+def linear(x_bf16, w, s_w) -> np.ndarray:
+    """Plain-epilogue FP8 projection: act_quant(x), then y = s_x*s_w*x_q.W^T.  [M, N]."""
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    w = _c(w, np.uint8)
+    M, K = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == K
+    out = np.zeros((M, N), dtype=np.float64)
+    lib.oracle_linear(_ptr(x), M, K, _ptr(w), float(s_w), N, _ptr(out))
+    return out
+
+
+def moe_linear(x_bf16, ids, w, s_w) -> np.ndarray:
+    """Grouped plain projection; w is [E, N, K] uint8, s_w [E] float32.  [T, N]."""
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    ids = _c(ids, np.int32)
+    w = _c(w, np.uint8)
+    s_w = _c(s_w, np.float32)
+    T, K = x.shape
+    E, N, K2 = w.shape
+    assert K2 == K and s_w.shape == (E,)
+    out = np.zeros((T, N), dtype=np.float64)
+    lib.oracle_moe_linear(_ptr(x), T, K, _ptr(ids), E, _ptr(w), _ptr(s_w), N, _ptr(out))
+    return out
+
+
+def add_rmsnorm(x_bf16, r_bf16, gamma_bf16, eps):
+    """Returns (h bf16 bits [M, K], y float64 [M, K]); r_bf16 may be None."""
+    lib = _load()
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    g = _c(gamma_bf16, np.uint16)
+    assert g.shape == (K,)
+    r = None if r_bf16 is None else _c(r_bf16, np.uint16)
+    if r is not None:
+        assert r.shape == x.shape
+    h = np.zeros((M, K), dtype=np.uint16)
+    y = np.zeros((M, K), dtype=np.float64)
+    lib.oracle_add_rmsnorm(_ptr(x), None if r is None else _ptr(r), _ptr(g), M, K, float(eps), _ptr(h), _ptr(y))
+    return h, y
+
+
+def quant_f32(y) -> tuple:
+    """Returns (xq uint8, s_x float32) of float32 values (shape kept)."""
+    lib = _load()
+    yf = _c(y, np.float32)
+    xq = np.zeros(yf.shape, dtype=np.uint8)
+    sx = np.zeros(1, dtype=np.float32)
+    lib.oracle_quant_f32(_ptr(yf), int(yf.size), _ptr(xq), _ptr(sx))
+    return xq, np.float32(sx[0])
+
+
+def add_rmsnorm_quant(x_bf16, r_bf16, gamma_bf16, eps):
+    """Residual add + RMSNorm + Quantize: (h bits, y float64, xq, s_x), the
+    quantisation taken on float32(y)."""
+    h, y = add_rmsnorm(x_bf16, r_bf16, gamma_bf16, eps)
+    xq, sx = quant_f32(y.astype(np.float32))
+    return h, y, xq, sx
 
 
 def decode_attn(q, q_stride, B, T, Hq, Hkv, d, k_cache, v_cache, seq_lens, scale) -> np.ndarray:

@@ -191,6 +191,70 @@ void oracle_moe_fc13_swiglu(const uint16_t* x, int T, int K, const int32_t* ids,
   }
 }
 
+void oracle_quant_f32(const float* y, long long n, uint8_t* xq, float* s_x) {
+  float amax = 0.0f;
+  for (long long i = 0; i < n; ++i) {
+    const float a = std::fabs(y[i]);
+    if (a > amax) amax = a;
+  }
+  if (amax == 0.0f) {
+    *s_x = 1.0f;
+    for (long long i = 0; i < n; ++i) xq[i] = 0;
+    return;
+  }
+  volatile float num = 448.0f;  // single IEEE roundings, as in oracle_act_quant
+  const float inv = num / amax;
+  *s_x = amax / num;
+  for (long long i = 0; i < n; ++i) {
+    volatile float prod = y[i] * inv;
+    xq[i] = oracle_f32_to_e4m3(prod);
+  }
+}
+
+void oracle_linear(const uint16_t* x, int M, int K, const uint8_t* w, float s_w, int N,
+                   double* out) {
+  std::vector<uint8_t> xq(static_cast<size_t>(M) * K);
+  float s_x = 0.0f;
+  oracle_act_quant(x, M, K, xq.data(), &s_x);
+  oracle_gemm_q(xq.data(), s_x, w, s_w, M, N, K, out);
+}
+
+void oracle_moe_linear(const uint16_t* x, int T, int K, const int32_t* ids, int E,
+                       const uint8_t* w, const float* s_w, int N, double* out) {
+  std::vector<uint8_t> xq(static_cast<size_t>(T) * K);
+  float s_x = 0.0f;
+  oracle_act_quant(x, T, K, xq.data(), &s_x);
+  for (int t = 0; t < T; ++t) {
+    const int e = ids[t];
+    double* row = out + static_cast<size_t>(t) * N;
+    if (e < 0 || e >= E) {
+      for (int n = 0; n < N; ++n) row[n] = std::nan("");
+      continue;
+    }
+    oracle_gemm_q(xq.data() + static_cast<size_t>(t) * K, s_x, w + static_cast<size_t>(e) * N * K,
+                  s_w[e], 1, N, K, row);
+  }
+}
+
+void oracle_add_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* gamma, int M,
+                        int K, float eps, uint16_t* h_out, double* y) {
+  std::vector<double> h(static_cast<size_t>(K));
+  for (int m = 0; m < M; ++m) {
+    const size_t base = static_cast<size_t>(m) * K;
+    double ss = 0.0;
+    for (int k = 0; k < K; ++k) {
+      // the residual stream is bf16: the exact sum is rounded once to bf16
+      uint16_t hb = x[base + k];
+      if (r != nullptr) hb = oracle_f64_to_bf16(oracle_bf16_to_f64(x[base + k]) + oracle_bf16_to_f64(r[base + k]));
+      h_out[base + k] = hb;
+      h[k] = oracle_bf16_to_f64(hb);
+      ss += h[k] * h[k];
+    }
+    const double inv_rms = 1.0 / std::sqrt(ss / K + static_cast<double>(eps));
+    for (int k = 0; k < K; ++k) y[base + k] = h[k] * inv_rms * oracle_bf16_to_f64(gamma[k]);
+  }
+}
+
 void oracle_attn_partial(const uint16_t* q, long long q_stride, int T, int Hq, int Hkv,
                          int d, const uint16_t* k, const uint16_t* v, int Lcap,
                          int b, int t, int h, int L, float scale, int key_lo, int key_hi,

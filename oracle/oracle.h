@@ -86,6 +86,34 @@ void oracle_fc_qkv_scale(const uint16_t* x, int M, int K, const uint8_t* w, floa
 void oracle_moe_fc13_swiglu(const uint16_t* x, int T, int K, const int32_t* ids, int E,
                             const uint8_t* w, const float* s_w, int N2, double* out);
 
+/* ---- Plain-epilogue projections (attention output projection, FC2 down
+ * projection): [NV] "CUDA kernel optimisation and fusion" lists the layer's
+ * GEMMs as FP8 weight-streaming GEMMs; without a fused epilogue the output is
+ * y itself.  oracle_linear: out[m][n] = y[m][n] of act_quant(x) and w [N][K].
+ * oracle_moe_linear: one activation scale over all T tokens, token t uses
+ * expert ids[t] (block w + ids[t]*N*K, scale s_w[ids[t]]); out is [T][N] in
+ * token order, a NaN row for an id outside [0, E). */
+void oracle_linear(const uint16_t* x, int M, int K, const uint8_t* w, float s_w, int N,
+                   double* out);
+void oracle_moe_linear(const uint16_t* x, int T, int K, const int32_t* ids, int E,
+                       const uint8_t* w, const float* s_w, int N, double* out);
+
+/* ---- Residual add + RMSNorm, the producer of the next GEMM's input ---------
+ * [XZY] "CUDA 内核优化与融合" / "运算融合" and [NV] "CUDA kernel optimisation and
+ * fusion" fuse (AllReduce +) RMSNorm + Quantize into one kernel ahead of the
+ * FP8 GEMM; on one GPU the AllReduce is absent and the residual add remains.
+ * Readings (the pages give no formula): the residual stream is bf16, so
+ *   h = bf16_rne(x + r)   (h = x when r is NULL), written to h_out;
+ *   y[m][k] = h[m][k] / sqrt(mean_k h[m][k]^2 + eps) * gamma[k]   (double).
+ * The Quantize step then takes y in the kernel's precision: oracle_quant_f32
+ * of (float)y. */
+void oracle_add_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* gamma, int M,
+                        int K, float eps, uint16_t* h_out, double* y);
+/* Per-tensor dynamic quantisation of float values, the rule of oracle_act_quant
+ * applied to fp32 inputs: amax = max|y|, inv = 448f/amax, s_x = amax/448f,
+ * xq = e4m3_rne_sat(y * inv) (one float rounding for the product). */
+void oracle_quant_f32(const float* y, long long n, uint8_t* xq, float* s_x);
+
 /* ---- A3: grouped-query decode attention, computed unsplit ----------------
  * [XZY] "Attention内核并行优化"; [NV] "CUDA kernel optimisation and fusion".
  * q[b][t][h][i] sits at q[(b*T + t)*q_stride + h*d + i]; K and V caches are

@@ -407,3 +407,127 @@ def test_moe_equals_per_token_dense_with_shared_scale():
     # a token routed elsewhere gives a different row (the expert id matters)
     other = (ids[0] + 1) % E
     assert not np.allclose(out[0], oracle.fc13_swiglu_q(xq[:1], sx, w[other], s_w[other])[0])
+
+
+# ------------------------------------------- plain projections (o_proj, FC2) --
+
+def test_linear_equals_unit_scaled_qkv_and_one_hot_column():
+    g = np.random.default_rng(61)
+    M, K, N = 3, 256, 160
+    x = dg.bf16_normal(g, (M, K))
+    w, s_w = dg.e4m3_weight(g, N, K)
+    # the QKV entry with q_scale = 1 is the plain projection (N = (Hq + 2Hkv) d)
+    assert np.array_equal(oracle.linear(x, w, s_w), oracle.fc_qkv_scale(x, w, s_w, 6, 2, 16, 1.0))
+    # one-hot input selects column k of W, times the known scales
+    xo = np.zeros((1, K), dtype=np.float32)
+    xo[0, 77] = -2.0
+    y = oracle.linear(dg.bf16_bits(xo), w, s_w)
+    expect = float(np.float32(2.0) / np.float32(448.0)) * float(s_w) * -448.0 * _dequant_torch(w[:, 77])
+    assert np.array_equal(y[0], expect)
+
+
+def test_moe_linear_equals_per_token_projection_with_shared_scale():
+    g = np.random.default_rng(62)
+    T, K, N, E = 7, 128, 64, 4
+    x = dg.bf16_normal(g, (T, K))
+    ws, scales = zip(*(dg.e4m3_weight(g, N, K) for _ in range(E)))
+    w = np.stack(ws)
+    s_w = np.array(scales, dtype=np.float32)
+    ids = np.array([3, 0, 3, 1, 2, 0, 3], dtype=np.int32)
+    out = oracle.moe_linear(x, ids, w, s_w)
+    xq, sx = oracle.act_quant(x)
+    xd, = (_dequant_torch(xq),)
+    for t in range(T):
+        ref = xd[t] @ _dequant_torch(w[ids[t]]).T * float(sx) * float(s_w[ids[t]])
+        assert np.allclose(out[t], ref, rtol=1e-12, atol=1e-14)
+    bad = oracle.moe_linear(x, np.array([0, 9, 0, 0, 0, 0, 0], dtype=np.int32), w, s_w)
+    assert np.isnan(bad[1]).all() and not np.isnan(bad[0]).any()
+
+
+# ------------------------------------------ residual add + RMSNorm + quant --
+
+def test_add_rmsnorm_quant_hand_example(golden_dir):
+    gold = json.load(open(os.path.join(golden_dir, "add_rmsnorm_quant_hand.json")))
+    x = _bits_of(gold["x"])
+    r = _bits_of(gold["r"])
+    gam = _bits_of(gold["gamma"])
+    h, y, xq, sx = oracle.add_rmsnorm_quant(x, r, gam, gold["eps"])
+    assert np.array_equal(h, _bits_of(gold["h"]))
+    assert y[0].tolist() == gold["y_row0"]
+    assert xq[0].tolist() == gold["xq_row0"]
+    assert sx == np.float32(1.0) / np.float32(112.0)
+
+
+def test_rmsnorm_matches_torch_rms_norm():
+    g = np.random.default_rng(63)
+    M, K = 5, 640
+    x = dg.bf16_normal(g, (M, K))
+    gam = dg.bf16_normal(g, (K,), std=0.5)
+    for eps in (1e-5, 0.25):
+        h, y = oracle.add_rmsnorm(x, None, gam, eps)
+        assert np.array_equal(h, x)  # no residual: h is x
+        ref = torch.nn.functional.rms_norm(torch.from_numpy(_bf16_torch(x)), (K,),
+                                           weight=torch.from_numpy(_bf16_torch(gam)), eps=float(np.float32(eps)))
+        assert np.allclose(y, ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_residual_add_matches_torch_bf16_add_and_norm_uses_the_rounded_sum():
+    g = np.random.default_rng(64)
+    M, K = 3, 512
+    x = dg.bf16_normal(g, (M, K))
+    r = dg.bf16_normal(g, (M, K), std=3.0)
+    gam = dg.bf16_bits(np.ones(K, dtype=np.float32))
+    h, y = oracle.add_rmsnorm(x, r, gam, 1e-6)
+    tx = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+    tr = torch.from_numpy(r.view(np.int16)).view(torch.bfloat16)
+    assert np.array_equal(h, (tx + tr).view(torch.int16).numpy().view(np.uint16))
+    # the norm is taken of h (the rounded sum): normalising h itself gives y
+    h2, y2 = oracle.add_rmsnorm(h, None, gam, 1e-6)
+    assert np.array_equal(h2, h) and np.array_equal(y2, y)
+
+
+def test_rmsnorm_invariants():
+    g = np.random.default_rng(65)
+    M, K = 4, 256
+    x = dg.bf16_normal(g, (M, K))
+    one = dg.bf16_bits(np.ones(K, dtype=np.float32))
+    _, y = oracle.add_rmsnorm(x, None, one, 0.0)
+    assert np.allclose((y ** 2).mean(axis=1), 1.0, rtol=1e-13)  # unit gain, eps = 0: unit mean square
+    xs = dg.bf16_bits(_bf16_torch(x).astype(np.float32) * np.float32(8.0))  # exact power-of-two scaling
+    _, ys = oracle.add_rmsnorm(xs, None, one, 0.0)
+    assert np.allclose(ys, y, rtol=1e-14, atol=0)
+    _, yp = oracle.add_rmsnorm(x[::-1].copy(), None, one, 0.0)  # rows are independent
+    assert np.array_equal(yp, y[::-1])
+    # a constant row c gives sign(c) * gamma; gamma enters per column
+    gam = dg.bf16_normal(g, (K,))
+    c = dg.bf16_bits(np.full((1, K), -3.0, dtype=np.float32))
+    _, yc = oracle.add_rmsnorm(c, None, gam, 0.0)
+    assert np.array_equal(yc[0], -_bf16_torch(gam))
+    # a zero row with eps > 0 normalises to zero, not NaN
+    _, yz = oracle.add_rmsnorm(np.zeros((1, K), dtype=np.uint16), None, gam, 1e-6)
+    assert not yz.any()
+
+
+def test_quant_f32_reduces_to_act_quant_on_bf16_values():
+    g = np.random.default_rng(66)
+    x = dg.bf16_normal(g, (3, 384))
+    xq, sx = oracle.act_quant(x)
+    xq2, sx2 = oracle.quant_f32(_bf16_torch(x).astype(np.float32))
+    assert sx2 == sx and np.array_equal(xq2, xq)
+    z, sz = oracle.quant_f32(np.zeros(10, dtype=np.float32))
+    assert sz == 1.0 and not z.any()
+
+
+def test_quant_f32_codes_are_nearest_by_brute_force():
+    g = np.random.default_rng(67)
+    y = (g.standard_normal(300) * np.exp(g.uniform(-6, 3, 300))).astype(np.float32)
+    xq, sx = oracle.quant_f32(y)
+    inv = np.float32(448.0) / np.float32(np.abs(y).max())
+    assert sx == np.float32(np.abs(y).max()) / np.float32(448.0)
+    codes = np.arange(256, dtype=np.uint8)
+    vals = _dequant_torch(codes)
+    finite = ~np.isnan(vals)
+    for i in range(y.size):
+        p = float(np.float32(y[i] * inv))
+        best = np.min(np.abs(vals[finite] - p))
+        assert abs(vals[xq[i]] - p) == best, (i, p, vals[xq[i]])
