@@ -62,6 +62,7 @@ def _load():
             "oracle_moe_linear": (None, [_P, _I, _I, _P, _I, _P, _P, _I, _P]),
             "oracle_add_rmsnorm": (None, [_P, _P, _P, _I, _I, _F, _P, _P]),
             "oracle_quant_f32": (None, [_P, _LL, _P, _P]),
+            "oracle_spec_verify_greedy": (None, [_P, _I, _I, _I, _P, _P, _P, _P]),
             "oracle_decode_attn": (None, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _P]),
             "oracle_attn_partial": (None, [_P, _LL, _I, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I,
                                            _F, _I, _I, _P, _P, _P]),
@@ -267,6 +268,20 @@ def add_rmsnorm_quant(x_bf16, r_bf16, gamma_bf16, eps):
     h, y = add_rmsnorm(x_bf16, r_bf16, gamma_bf16, eps)
     xq, sx = quant_f32(y.astype(np.float32))
     return h, y, xq, sx
+
+
+def spec_verify_greedy(logits_bf16, draft):
+    """logits [B, T, V] bf16 bits, draft [B, T-1] int32 ->
+    (target_ids [B, T], n_accepted [B], emitted [B, T]) int32."""
+    lib = _load()
+    lg = _c(logits_bf16, np.uint16)
+    B, T, V = lg.shape
+    dr = _c(draft, np.int32).reshape(B, T - 1)
+    tid = np.zeros((B, T), dtype=np.int32)
+    nacc = np.zeros(B, dtype=np.int32)
+    em = np.zeros((B, T), dtype=np.int32)
+    lib.oracle_spec_verify_greedy(_ptr(lg), B, T, V, _ptr(dr), _ptr(tid), _ptr(nacc), _ptr(em))
+    return tid, nacc, em
 
 
 def decode_attn(q, q_stride, B, T, Hq, Hkv, d, k_cache, v_cache, seq_lens, scale) -> np.ndarray:

@@ -255,6 +255,33 @@ void oracle_add_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* ga
   }
 }
 
+void oracle_spec_verify_greedy(const uint16_t* logits, int B, int T, int V, const int32_t* draft,
+                               int32_t* target_ids, int32_t* n_accepted, int32_t* emitted) {
+  for (int b = 0; b < B; ++b) {
+    // the token the target model itself would emit after each input position
+    for (int t = 0; t < T; ++t) {
+      const uint16_t* row = logits + (static_cast<size_t>(b) * T + t) * static_cast<size_t>(V);
+      int best = 0;
+      double best_v = oracle_bf16_to_f64(row[0]);
+      for (int v = 1; v < V; ++v) {
+        const double x = oracle_bf16_to_f64(row[v]);
+        if (x > best_v) {  // strict: the lowest index wins a tie
+          best_v = x;
+          best = v;
+        }
+      }
+      target_ids[static_cast<size_t>(b) * T + t] = best;
+    }
+    // drafts are accepted while they equal the target's own token; the first
+    // mismatch ends the run and the target's token there is emitted instead
+    int n = 0;
+    while (n < T - 1 && draft[static_cast<size_t>(b) * (T - 1) + n] == target_ids[static_cast<size_t>(b) * T + n]) ++n;
+    n_accepted[b] = n;
+    for (int t = 0; t < T; ++t)
+      emitted[static_cast<size_t>(b) * T + t] = t <= n ? target_ids[static_cast<size_t>(b) * T + t] : -1;
+  }
+}
+
 void oracle_attn_partial(const uint16_t* q, long long q_stride, int T, int Hq, int Hkv,
                          int d, const uint16_t* k, const uint16_t* v, int Lcap,
                          int b, int t, int h, int L, float scale, int key_lo, int key_hi,

@@ -114,6 +114,21 @@ void oracle_add_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* ga
  * xq = e4m3_rne_sat(y * inv) (one float rounding for the product). */
 void oracle_quant_f32(const float* y, long long n, uint8_t* xq, float* s_x);
 
+/* ---- Greedy speculative verification on the device ([XZY] "推测解码",
+ * "端到端的工作流" and "通过 CUDA Graph 和重叠调度器减少主机端开销"; [NV]
+ * speculative-decoding section) ----------------------------------------------
+ * The target step reads T inputs per sequence: the last accepted token, then
+ * the T-1 draft tokens draft[b][0..T-2].  logits [B][T][V] (bf16) are the
+ * target's outputs at those positions.  Readings: the token the target itself
+ * would generate is the greedy argmax (lowest index on a tie); draft[b][i] is
+ * accepted while it equals target_ids[b][i] for every earlier i; at the first
+ * mismatch the target's own token is emitted instead, and with no mismatch the
+ * token after the last draft is emitted as well.
+ *   target_ids [B][T]; n_accepted[b] = accepted drafts (0..T-1);
+ *   emitted [B][T] = target_ids[b][0..n] followed by -1 (n + 1 tokens). */
+void oracle_spec_verify_greedy(const uint16_t* logits, int B, int T, int V, const int32_t* draft,
+                               int32_t* target_ids, int32_t* n_accepted, int32_t* emitted);
+
 /* ---- A3: grouped-query decode attention, computed unsplit ----------------
  * [XZY] "Attention内核并行优化"; [NV] "CUDA kernel optimisation and fusion".
  * q[b][t][h][i] sits at q[(b*T + t)*q_stride + h*d + i]; K and V caches are

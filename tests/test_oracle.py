@@ -531,3 +531,50 @@ def test_quant_f32_codes_are_nearest_by_brute_force():
         p = float(np.float32(y[i] * inv))
         best = np.min(np.abs(vals[finite] - p))
         assert abs(vals[xq[i]] - p) == best, (i, p, vals[xq[i]])
+
+
+# ------------------------------------------------ speculative verification --
+
+def test_spec_verify_hand_example(golden_dir):
+    gold = json.load(open(os.path.join(golden_dir, "spec_verify_hand.json")))
+    T, V = len(gold["hot"]), gold["V"]
+    lg = np.zeros((1, T, V), dtype=np.float32)
+    for t, v in enumerate(gold["hot"]):
+        lg[0, t, v] = 1.0
+    tid, nacc, em = oracle.spec_verify_greedy(dg.bf16_bits(lg), np.array([gold["draft"]], dtype=np.int32))
+    assert tid[0].tolist() == gold["target_ids"]
+    assert int(nacc[0]) == gold["n_accepted"]
+    assert em[0].tolist() == gold["emitted"]
+
+
+def test_spec_verify_matches_numpy_argmax_and_brute_force_acceptance():
+    g = np.random.default_rng(71)
+    B, T, V = 6, 4, 1000
+    lg = dg.bf16_normal(g, (B, T, V))
+    lg[0, 1, 7] = lg[0, 1, 9] = dg.bf16_bits(np.float32([50.0]))[0]  # a tie: the lower index wins
+    ref = np.argmax(_bf16_torch(lg), axis=2)  # numpy returns the first maximal index
+    assert ref[0, 1] == 7
+    draft = g.integers(0, V, size=(B, T - 1)).astype(np.int32)
+    # plant accept runs of every length 0..T-1
+    for b, n in enumerate([0, 1, 2, 3, 3, 1]):
+        draft[b, :n] = ref[b, :n]
+        if n < T - 1 and draft[b, n] == ref[b, n]:
+            draft[b, n] = (ref[b, n] + 1) % V
+    tid, nacc, em = oracle.spec_verify_greedy(lg, draft)
+    assert np.array_equal(tid, ref)
+    for b in range(B):
+        n = 0
+        for i in range(T - 1):  # brute force: longest matching prefix
+            if all(draft[b, j] == ref[b, j] for j in range(i + 1)):
+                n = i + 1
+        assert nacc[b] == n
+        assert em[b, :n + 1].tolist() == ref[b, :n + 1].tolist() and (em[b, n + 1:] == -1).all()
+    assert nacc.tolist() == [0, 1, 2, 3, 3, 1]
+
+
+def test_spec_verify_single_position_emits_one_token():
+    g = np.random.default_rng(72)
+    lg = dg.bf16_normal(g, (3, 1, 50))
+    tid, nacc, em = oracle.spec_verify_greedy(lg, np.zeros((3, 0), dtype=np.int32))
+    assert (nacc == 0).all() and np.array_equal(em[:, 0], tid[:, 0])
+    assert np.array_equal(tid[:, 0], np.argmax(_bf16_torch(lg)[:, 0], axis=1))
