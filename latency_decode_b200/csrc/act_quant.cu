@@ -9,8 +9,7 @@
 // One thread-block cluster of C <= 8 CTAs covers the whole [M][K] input: each
 // CTA reduces |x| over its slice, the cluster merges the C partial maxima
 // through distributed shared memory (no global round trip), and each CTA then
-// quantises its own slice.  The input (<= 1 MB) is read twice; the second read
-// hits L2.
+// quantises its own slice from registers (the input is read from memory once).
 #include <cuda_fp8.h>
 
 #include "dl_device.cuh"
@@ -62,19 +61,22 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
   const int v1 = static_cast<int>(static_cast<long long>(nv) * (r + 1) / C);
   const uint4* xv = reinterpret_cast<const uint4*>(x);
 
-  // eight independent 16-byte loads in flight per thread per round
-  constexpr int kBatch = 8;
+  // One pass over memory: this CTA's slice (<= kKeep vectors per thread, which
+  // covers M*K <= 8*512*12*8 = 393216 with 8 CTAs) is loaded once, all loads in
+  // flight together, and kept in registers for the quantisation after the
+  // cluster amax; larger inputs read the remainder twice.
+  constexpr int kKeep = 12;
+  uint4 u[kKeep];
   float m = 0.0f;
-  for (int base = v0 + threadIdx.x; base < v1; base += kBatch * kAqThreads) {
-    uint4 u[kBatch];
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
-      const int i = base + j * kAqThreads;
-      u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int j = 0; j < kBatch; ++j) m = fmaxf(m, absmax8(u[j]));
+  for (int j = 0; j < kKeep; ++j) {
+    const int i = v0 + threadIdx.x + j * kAqThreads;
+    u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
   }
+#pragma unroll
+  for (int j = 0; j < kKeep; ++j) m = fmaxf(m, absmax8(u[j]));
+  for (int i = v0 + threadIdx.x + kKeep * kAqThreads; i < v1; i += kAqThreads)  // larger inputs
+    m = fmaxf(m, absmax8(__ldg(xv + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
@@ -92,23 +94,16 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
   for (int p = 0; p < C; ++p) amax = fmaxf(amax, dsmem_ld_f32(dsmem_addr(local, p)));
 
   uint2* q2 = reinterpret_cast<uint2*>(xq);
-  if (amax > 0.0f) {
-    const float inv = __fdiv_rn(448.0f, amax);
-    for (int base = v0 + threadIdx.x; base < v1; base += kBatch * kAqThreads) {
-      uint4 u[kBatch];
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int i = base + j * kAqThreads;
-        u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int i = base + j * kAqThreads;
-        if (i < v1) q2[i] = make_uint2(quant4(u[j].x, u[j].y, inv), quant4(u[j].z, u[j].w, inv));
-      }
-    }
-  } else {
-    for (int i = v0 + threadIdx.x; i < v1; i += kAqThreads) q2[i] = make_uint2(0u, 0u);
+  for (int j = 0; j < kKeep; ++j) {
+    const int i = v0 + threadIdx.x + j * kAqThreads;
+    if (i < v1)
+      q2[i] = amax > 0.0f ? make_uint2(quant4(u[j].x, u[j].y, inv), quant4(u[j].z, u[j].w, inv)) : make_uint2(0u, 0u);
+  }
+  for (int i = v0 + threadIdx.x + kKeep * kAqThreads; i < v1; i += kAqThreads) {
+    const uint4 w = __ldg(xv + i);
+    q2[i] = amax > 0.0f ? make_uint2(quant4(w.x, w.y, inv), quant4(w.z, w.w, inv)) : make_uint2(0u, 0u);
   }
   if (r == 0 && threadIdx.x == 0) *s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 

@@ -186,6 +186,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   const uint8_t* wsrc = a.w + expert * a.w_expert_bytes +
                         (static_cast<long long>(tile) * a.KB + kb0) * SUBS * kSubBytes;
 
+  // The fused quantiser reads all of x right after the PDL wait: warm L2 with
+  // its lines now, while the CTA sets up (a hint only; x is read after the wait).
+  if (a.x != nullptr && warp >= 2) {
+    const char* xb = reinterpret_cast<const char*>(a.x);
+    const long long xbytes = static_cast<long long>(a.M) * a.K * 2;
+    for (long long off = static_cast<long long>(threadIdx.x - 64) * 128; off < xbytes; off += 64 * 128)
+      prefetch_l2_line(xb + off);
+  }
+
   // ---- barriers and Tensor Memory ---------------------------------------------------
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -310,14 +319,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
           keep[2 * j + 1] = __ldg(src + 1);
         }
       }
-      float m0 = 0.0f, m1 = 0.0f;
-      int i = t;
-      for (; i + 64 < nv; i += 128) {
-        m0 = fmaxf(m0, absmax8(__ldg(xv + i)));
-        m1 = fmaxf(m1, absmax8(__ldg(xv + i + 64)));
+      // amax over all of x: 16 independent 16-byte loads in flight per thread per
+      // round, so x (10 KB at batch 1) arrives in one memory round trip.
+      constexpr int kBatch = 16;
+      float m = 0.0f;
+      for (int base = t; base < nv; base += 64 * kBatch) {
+        uint4 u[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const int i = base + 64 * j;
+          u[j] = i < nv ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) m = fmaxf(m, absmax8(u[j]));
       }
-      if (i < nv) m0 = fmaxf(m0, absmax8(__ldg(xv + i)));
-      float m = fmaxf(m0, m1);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (lane == 0) misc->wmax[warp - 2] = m;
