@@ -63,6 +63,7 @@ def _load():
             "oracle_add_rmsnorm": (None, [_P, _P, _P, _I, _I, _F, _P, _P]),
             "oracle_quant_f32": (None, [_P, _LL, _P, _P]),
             "oracle_spec_verify_greedy": (None, [_P, _I, _I, _I, _P, _P, _P, _P]),
+            "oracle_decode_attn_fp8kv": (None, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _F, _F, _P]),
             "oracle_decode_attn": (None, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _P]),
             "oracle_attn_partial": (None, [_P, _LL, _I, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I,
                                            _F, _I, _I, _P, _P, _P]),
@@ -297,6 +298,21 @@ def decode_attn(q, q_stride, B, T, Hq, Hkv, d, k_cache, v_cache, seq_lens, scale
     out = np.zeros((B, T, Hq, d), dtype=np.float64)
     lib.oracle_decode_attn(_ptr(q), int(q_stride), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap,
                            _ptr(sl), float(scale), _ptr(out))
+    return out
+
+
+def decode_attn_fp8kv(q, q_stride, B, T, Hq, Hkv, d, k_codes, v_codes, seq_lens, scale, s_k, s_v) -> np.ndarray:
+    """As decode_attn, with e4m3 caches (uint8 [B, Hkv, Lcap, d]) and per-tensor scales."""
+    lib = _load()
+    q = _c(q, np.uint16)
+    k = _c(k_codes, np.uint8)
+    v = _c(v_codes, np.uint8)
+    sl = _c(seq_lens, np.int32)
+    Lcap = k.shape[2]
+    assert k.shape == (B, Hkv, Lcap, d) and v.shape == k.shape and sl.shape == (B,)
+    out = np.zeros((B, T, Hq, d), dtype=np.float64)
+    lib.oracle_decode_attn_fp8kv(_ptr(q), int(q_stride), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(sl),
+                                 float(scale), float(s_k), float(s_v), _ptr(out))
     return out
 
 

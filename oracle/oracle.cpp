@@ -340,6 +340,42 @@ void oracle_decode_attn(const uint16_t* q, long long q_stride, int B, int T, int
   }
 }
 
+void oracle_decode_attn_fp8kv(const uint16_t* q, long long q_stride, int B, int T, int Hq, int Hkv,
+                              int d, const uint8_t* k, const uint8_t* v, int Lcap,
+                              const int32_t* seq_lens, float scale, float s_k, float s_v,
+                              double* out) {
+  const int g = Hq / Hkv;
+  std::vector<double> qd(static_cast<size_t>(d)), s, o(static_cast<size_t>(d));
+  for (int b = 0; b < B; ++b) {
+    const int L = seq_lens[b];
+    for (int t = 0; t < T; ++t) {
+      for (int h = 0; h < Hq; ++h) {
+        const uint16_t* qr = q + (static_cast<long long>(b) * T + t) * q_stride + static_cast<long long>(h) * d;
+        const size_t head = (static_cast<size_t>(b) * Hkv + h / g) * static_cast<size_t>(Lcap) * d;
+        for (int i = 0; i < d; ++i) qd[i] = oracle_bf16_to_f64(qr[i]);
+        const int visible = L - T + t + 1;  // keys 0 .. L-T+t
+        s.assign(static_cast<size_t>(visible > 0 ? visible : 0), 0.0);
+        double mx = -std::numeric_limits<double>::infinity();
+        for (int j = 0; j < visible; ++j) {
+          double dot = 0.0;  // the cache holds k = s_k * e4m3(code)
+          for (int i = 0; i < d; ++i) dot += qd[i] * (static_cast<double>(s_k) * kE4m3.v[k[head + static_cast<size_t>(j) * d + i]]);
+          s[j] = static_cast<double>(scale) * dot;
+          mx = s[j] > mx ? s[j] : mx;
+        }
+        double l = 0.0;
+        for (int i = 0; i < d; ++i) o[i] = 0.0;
+        for (int j = 0; j < visible; ++j) {
+          const double p = std::exp(s[j] - mx);
+          l += p;
+          for (int i = 0; i < d; ++i) o[i] += p * (static_cast<double>(s_v) * kE4m3.v[v[head + static_cast<size_t>(j) * d + i]]);
+        }
+        double* dst = out + ((static_cast<size_t>(b) * T + t) * Hq + h) * d;
+        for (int i = 0; i < d; ++i) dst[i] = l > 0.0 ? o[i] / l : 0.0;
+      }
+    }
+  }
+}
+
 void oracle_lse_combine(int S, const double* m, const double* l, const double* o_parts,
                         int d, double* out) {
   double mstar = -std::numeric_limits<double>::infinity();

@@ -140,6 +140,16 @@ void oracle_decode_attn(const uint16_t* q, long long q_stride, int B, int T, int
                         int Hkv, int d, const uint16_t* k, const uint16_t* v, int Lcap,
                         const int32_t* seq_lens, float scale, double* out);
 
+/* ---- A3 with an FP8 KV cache ([TC] and [XZY]: FP8 is used for attention as
+ * well as for the GEMMs and MoE).  Reading: the cache holds e4m3 codes with one
+ * per-tensor scale each for K and V, k = s_k * e4m3(code), v = s_v * e4m3(code);
+ * q stays bf16.  Otherwise exactly oracle_decode_attn (same layout, GQA map and
+ * bottom-right causal rule); k and v are [B][Hkv][Lcap][d] bytes. */
+void oracle_decode_attn_fp8kv(const uint16_t* q, long long q_stride, int B, int T, int Hq, int Hkv,
+                              int d, const uint8_t* k, const uint8_t* v, int Lcap,
+                              const int32_t* seq_lens, float scale, float s_k, float s_v,
+                              double* out);
+
 /* Partial softmax state of one (b, q head, query t) over the visible keys that
  * fall in [key_lo, key_hi): m = max logit (-inf if none), l = sum exp(s - m),
  * o = sum exp(s - m) v (unnormalised, length d).  Used only to check the

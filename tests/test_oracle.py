@@ -578,3 +578,39 @@ def test_spec_verify_single_position_emits_one_token():
     tid, nacc, em = oracle.spec_verify_greedy(lg, np.zeros((3, 0), dtype=np.int32))
     assert (nacc == 0).all() and np.array_equal(em[:, 0], tid[:, 0])
     assert np.array_equal(tid[:, 0], np.argmax(_bf16_torch(lg)[:, 0], axis=1))
+
+
+# ------------------------------------------------------ FP8 KV attention --
+
+def test_fp8kv_attention_equals_bf16_attention_on_exactly_representable_caches():
+    """With power-of-two scales every s * e4m3 value is exact in bf16, so the
+    FP8-cache attention must equal the (pinned) bf16 attention on those values."""
+    g = np.random.default_rng(81)
+    B, T, Hq, Hkv, d, Lcap = 2, 4, 8, 2, 64, 96
+    q = dg.bf16_normal(g, (B, T, Hq, d))
+    kc = g.integers(0, 256, size=(B, Hkv, Lcap, d)).astype(np.uint8)
+    vc = g.integers(0, 256, size=(B, Hkv, Lcap, d)).astype(np.uint8)
+    kc[(kc & 0x7F) == 0x7F] = 0x30  # no NaN codes
+    vc[(vc & 0x7F) == 0x7F] = 0x38
+    s_k, s_v = np.float32(2.0 ** -7), np.float32(2.0 ** -5)
+    sl = np.int32([96, 37])
+    got = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.125, s_k, s_v)
+    kb = dg.bf16_bits((_dequant_torch(kc) * float(s_k)).astype(np.float32))
+    vb = dg.bf16_bits((_dequant_torch(vc) * float(s_v)).astype(np.float32))
+    assert np.array_equal(_bf16_torch(kb), _dequant_torch(kc) * float(s_k))  # exact in bf16
+    ref = oracle.decode_attn(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kb, vb, sl, 0.125)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_fp8kv_scales_enter_as_stated():
+    """s_v scales the output linearly; s_k acts as a softmax temperature
+    (s_k * scale is all that matters)."""
+    g = np.random.default_rng(82)
+    B, T, Hq, Hkv, d, Lcap = 1, 1, 4, 1, 64, 50
+    q = dg.bf16_normal(g, (B, T, Hq, d))
+    kc = g.integers(0, 0x7E, size=(B, Hkv, Lcap, d)).astype(np.uint8)
+    vc = g.integers(0, 0x7E, size=(B, Hkv, Lcap, d)).astype(np.uint8)
+    sl = np.int32([50])
+    a = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.5, 0.01, 1.0)
+    b = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.25, 0.02, 3.0)
+    assert np.allclose(b, 3.0 * a, rtol=1e-12)
