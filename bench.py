@@ -42,6 +42,9 @@ def parse_args():
     p.add_argument("--replicas", type=int, default=0, help="layer copies to rotate through (0 = auto)")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline sample length")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-full-layer", action="store_true", help="skip the whole-layer (7-kernel) figure")
+    p.add_argument("--profile-steps", type=int, default=0,
+                   help="only run this many direct-launch layer steps (for a profiler), print no JSON line")
     return p.parse_args()
 
 
@@ -256,6 +259,40 @@ def make_layers(wl, R, seed_base, device, cluster):
     return layers, kvs, xs, seq_lens, sl
 
 
+def make_full_layers(wl, R, seed_base, device, cluster):
+    """R independent whole pre-norm layers (QKV, attention, O_proj, FC13, FC2,
+    two RMSNorms), random weights of the workload's shapes drawn on the device."""
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200.layer import FullDecodeLayer
+    out = []
+    for r in range(R):
+        gen = torch.Generator(device=device).manual_seed(seed_base + r)
+        wq, sq = dg.e4m3_weight_torch(gen, wl.n_qkv, wl.K, device)
+        wo, so = dg.e4m3_weight_torch(gen, wl.K, wl.k_o, device)
+        w13, s13 = dg.e4m3_weight_torch(gen, wl.N2, wl.K, device)
+        w2, s2 = dg.e4m3_weight_torch(gen, wl.K, wl.k_fc2, device)
+        gains = [(1.0 + 0.1 * torch.randn(wl.K, generator=gen, device=device)).to(torch.bfloat16).view(torch.int16)
+                 for _ in range(2)]
+        lay = FullDecodeLayer(wq, sq, wo, so, w13, s13, w2, s2, gains[0], gains[1], Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d,
+                              q_scale=1.0 / math.sqrt(wl.d), M=wl.M, B=wl.B, T=wl.T, cluster=cluster,
+                              device=device)
+        del wq, wo, w13, w2
+        kc = torch.randn((wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device).to(torch.bfloat16)
+        vc = torch.randn((wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device).to(torch.bfloat16)
+        x = torch.randn((wl.M, wl.K), generator=gen, device=device).to(torch.bfloat16)
+        hres = torch.randn((wl.M, wl.K), generator=gen, device=device).to(torch.bfloat16)
+        out.append((lay, kc.view(torch.int16), vc.view(torch.int16), x.view(torch.int16), hres.view(torch.int16)))
+    torch.cuda.synchronize()
+    return out
+
+
+def gemm_launches(M, K):
+    """Kernels one GEMM entry point launches: the GEMM quantises inputs of up to
+    32768 elements itself, larger ones get a quantise kernel first."""
+    return 1 if M * K <= 32768 else 2
+
+
 def timed(fn, steps, stream):
     import torch
     start = torch.cuda.Event(enable_timing=True)
@@ -299,6 +336,15 @@ def run_ours(args):
         r = i % R
         layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens,
                        stream=torch.cuda.current_stream().cuda_stream, flags=flags)
+
+    if args.profile_steps > 0:  # a short, graph-free run of the chain for a profiler
+        for i in range(args.profile_steps):
+            step(i)
+        for lay in layers:
+            lay.read_status(h)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     for i in range(max(args.warmup, 3)):
         step(i)
@@ -399,9 +445,10 @@ def run_ours(args):
                                    stream=torch.cuda.current_stream().cuda_stream))
 
     kv_bytes = int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
+    gl = gemm_launches(wl.M, K)
     fam = {
-        "fc13_swiglu": (call_fc13, wl.N2 * wl.K, 2),
-        "fc_qkv_scale": (call_qkv, wl.n_qkv * wl.K, 2),
+        "fc13_swiglu": (call_fc13, wl.N2 * wl.K, gl),
+        "fc_qkv_scale": (call_qkv, wl.n_qkv * wl.K, gl),
         "decode_attn": (call_attn, kv_bytes, 1),
     }
     peak, peak_kind = peak_hbm()
@@ -423,30 +470,62 @@ def run_ours(args):
     for lay in layers:
         lay.read_status(h)
 
+    # ---- the whole pre-norm layer (adds O_proj, FC2 and both RMSNorm producers) ----
+    full = None
+    if not args.no_full_layer:
+        fbytes = wl.n_qkv * K + wl.K * wl.k_o + wl.N2 * K + wl.K * wl.k_fc2
+        RF = max(2, math.ceil(3 * L2_BYTES / (fbytes + 2 * wl.B * wl.Hkv * wl.Lcap * wl.d * 2)))
+        fl = make_full_layers(wl, RF, 5000 * (rank + 1), device, cluster)
+
+        def full_step(i):
+            lay, kc, vc, x, hres = fl[i % RF]
+            lay.step(x, hres, kc, vc, seq_lens, stream=torch.cuda.current_stream().cuda_stream)
+
+        for i in range(3):
+            full_step(i)
+        GF = RF * max(1, 24 // RF)
+        fmode = "direct"
+        try:
+            gbig, gs = capture(full_step, range(GF)), [capture(full_step, [r]) for r in range(RF)]
+            graph_steps(6, gbig, gs, GF)
+            us_full = timed_graph(args.steps, gbig, gs, GF) * 1e3 / args.steps
+            fmode = "graph"
+            del gbig, gs
+        except Exception:
+            us_full = timed(full_step, args.steps, stream) * 1e3 / args.steps
+        for entry in fl:
+            entry[0].read_status(h)
+        us_full = max_over_ranks(us_full)
+        # norm1, QKV (x_q from the norm), attention, O_proj, norm2, FC13 (x_q from the norm), FC2
+        f_launches = 1 + 1 + 1 + gemm_launches(wl.M, wl.k_o) + 1 + 1 + gemm_launches(wl.M, wl.k_fc2)
+        full = {"us": us_full, "alg_bytes": fbytes + kv_bytes,
+                "achieved_gbs": (fbytes + kv_bytes) / (us_full * 1e-6) / 1e9,
+                "frac": (fbytes + kv_bytes) / (us_full * 1e-6) / 1e9 / peak,
+                "launches_per_step": f_launches, "mode": fmode, "replicas": RF,
+                "steps": "add+RMSNorm+quant -> FC_QKV -> attention -> O_proj -> add+RMSNorm+quant -> FC13+SwiGLU "
+                         "-> FC2"}
+        del fl
+        torch.cuda.empty_cache()
+
     # ---- end to end through the public API with host buffers ----
-    r0 = 0
-    hx1 = torch.empty_like(xs[0][0], device="cpu").pin_memory()
-    hx2 = torch.empty_like(xs[0][1], device="cpu").pin_memory()
-    hx1.copy_(xs[0][0].cpu())
-    hx2.copy_(xs[0][1].cpu())
-    ha = torch.empty_like(layers[0].attn_out, device="cpu").pin_memory()
-    hf = torch.empty_like(layers[0].ffn_out, device="cpu").pin_memory()
-    dx1 = [torch.empty_like(xs[r][0]) for r in range(R)]
-    dx2 = [torch.empty_like(xs[r][1]) for r in range(R)]
+    # The step's two activations travel in one pinned buffer and its two
+    # results come back in one (DecodeLayer keeps them contiguous): one copy
+    # each way per step.
+    hx = torch.stack([xs[0][0], xs[0][1]]).cpu().pin_memory()
+    hout = torch.empty_like(layers[0].out_buf, device="cpu").pin_memory()
+    dx = [torch.empty_like(hx, device=device) for _ in range(R)]
 
     def e2e_step(i):
         r = i % R
-        dx1[r].copy_(hx1, non_blocking=True)
-        dx2[r].copy_(hx2, non_blocking=True)
-        layers[r].step(dx1[r], dx2[r], kvs[r][0], kvs[r][1], seq_lens, stream=h)
-        ha.copy_(layers[r].attn_out, non_blocking=True)
-        hf.copy_(layers[r].ffn_out, non_blocking=True)
+        dx[r].copy_(hx, non_blocking=True)
+        layers[r].step(dx[r][0], dx[r][1], kvs[r][0], kvs[r][1], seq_lens, stream=h)
+        hout.copy_(layers[r].out_buf, non_blocking=True)
 
     for i in range(3):
         e2e_step(i)
     us_e2e = max_over_ranks(timed(e2e_step, args.steps, stream) * 1e3 / args.steps)
-    h2d = hx1.numel() * 2 + hx2.numel() * 2
-    d2h = ha.numel() * 2 + hf.numel() * 2
+    h2d = hx.numel() * 2
+    d2h = hout.numel() * 2
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -481,7 +560,8 @@ def run_ours(args):
         "layer_achieved_gbs": (wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes) / (us_layer * 1e-6) / 1e9,
         "e2e": {"value": us_e2e, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "cpu_baseline": cpu,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": (2 * gl + 1) * args.steps,
+        "full_layer": full,
         "clocks": clk,
         "replicas": R,
     }

@@ -43,7 +43,8 @@
  *     [8, 12)       float  s_x, the activation scale of the last GEMM call
  *     [256, 256+M*K) uint8 x_q, the e4m3 activations [M][K] of the last GEMM call
  *   Two calls that may run concurrently (or overlap under PDL) must not share
- *   a workspace.
+ *   a workspace, except dl_add_rmsnorm_quant and the GEMM that follows it with
+ *   DL_FLAG_XQ_READY, which hand x_q over through it.
  */
 #ifndef LATENCY_DECODE_DL_H
 #define LATENCY_DECODE_DL_H
@@ -71,6 +72,10 @@ typedef enum dl_status {
 #define DL_FLAG_DEBUG_TIMEOUT 2u  /* test hook: shortens every bounded wait to ~2 ms and
                                      withholds the last pipeline load, so the consumer's
                                      wait runs out and DL_ERR_TIMEOUT is reported */
+#define DL_FLAG_XQ_READY 4u        /* GEMM entry points: the workspace already holds x_q and
+                                     s_x, written into this same workspace by
+                                     dl_add_rmsnorm_quant; the GEMM skips its activation
+                                     quantisation and `x` may be NULL */
 #define DL_FLAG_SPLIT_SHIFT 8     /* bits [8,13): if non-zero, force the GEMM split-K
                                      cluster size (1..8), or the number of clusters per
                                      (b, kv head) of dl_decode_attn (1..16), instead of
@@ -188,6 +193,62 @@ dl_status dl_moe_fc13_swiglu_grouped(const uint16_t* x, int T, int K, const int3
                                      void* stream, unsigned flags);
 
 /* ---------------------------------------------------------------------------
+ * Plain-epilogue FP8 projection: the attention output projection and the FC2
+ * down projection of the layer.  [NV] "CUDA kernel optimisation and fusion"
+ * (the layer's GEMMs are low-latency FP8 weight-streaming GEMMs); [XZY]
+ * "CUDA 内核优化与融合" (FP8 GEMMs, Quantize fused ahead of them).
+ *   x        bf16 [M][K] (may be NULL with DL_FLAG_XQ_READY)
+ *   w_packed e4m3, DL_PACK_PLAIN layout of the [N][K] weight
+ *   out      bf16 [M][N], row-major
+ * out = bf16(s_x * s_w * x_q . W^T), accumulated in fp32 on the tensor cores,
+ * with x_q, s_x as for dl_fc13_swiglu (or taken from the workspace with
+ * DL_FLAG_XQ_READY).  Supported: 1 <= M <= 64, M*K <= 64*8192, K % 128 == 0,
+ * N % 128 == 0.
+ * ------------------------------------------------------------------------- */
+dl_status dl_gemm_e4m3(const uint16_t* x, int M, int K, const uint8_t* w_packed,
+                       const float* w_scale, int N, uint16_t* out, void* ws, size_t ws_bytes,
+                       void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * Grouped MoE expert projection with a plain epilogue (the expert FC2 down
+ * projection), top-1.  Same routing, arguments and rules as
+ * dl_moe_fc13_swiglu_grouped, with E consecutive DL_PACK_PLAIN blocks of N*K
+ * bytes and out bf16 [T][N] in token order.  Supported: 1 <= T <= 64,
+ * T*K <= 64*8192, 1 <= E <= 1024, K % 128 == 0, N % 128 == 0.
+ * ------------------------------------------------------------------------- */
+dl_status dl_moe_gemm_grouped(const uint16_t* x, int T, int K, const int32_t* expert_ids, int E,
+                              const uint8_t* w_packed, const float* w_scales, int N,
+                              uint16_t* out, void* ws, size_t ws_bytes, void* stream,
+                              unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * Residual add + RMSNorm + Quantize, one kernel producing the FP8 input of the
+ * next GEMM.  [XZY] "CUDA 内核优化与融合", item "运算融合", and [NV] "CUDA
+ * kernel optimisation and fusion" fuse (AllReduce +) RMSNorm + Quantize; on
+ * one GPU the AllReduce is absent and the residual add takes its place.
+ *   x         bf16 [M][K], the sub-layer output (or the hidden state)
+ *   residual  bf16 [M][K] or NULL
+ *   h_out     bf16 [M][K] or NULL; receives h = bf16_rne(x + residual)
+ *             (h = x when residual is NULL).  It may be x or residual itself
+ *             (in-place update) but must not partially overlap either.
+ *   gamma     bf16 [K], the RMSNorm gain
+ *   eps       > 0
+ *   ws        the workspace of the GEMM that consumes the result (at least
+ *             dl_workspace_bytes(M, K)); x_q [M][K] and s_x are written there.
+ * Per token row: y = (h * rsqrt(mean(h^2) + eps)) * gamma in fp32; then one
+ * per-tensor scale s_x = max|y| / 448 and x_q = e4m3(y * (448 / max|y|)), as
+ * in the GEMMs' own quantisation.  Run the consuming GEMM next on the same
+ * stream with DL_FLAG_XQ_READY and the same ws: these two calls share the
+ * workspace by design (under DL_FLAG_PDL the GEMM reads x_q only after it
+ * waited for this kernel).
+ * Supported: 1 <= M <= 64, M*K <= 64*8192, K % 128 == 0; pointers 16-byte
+ * aligned.
+ * ------------------------------------------------------------------------- */
+dl_status dl_add_rmsnorm_quant(const uint16_t* x, const uint16_t* residual, uint16_t* h_out,
+                               const uint16_t* gamma, int M, int K, float eps, void* ws,
+                               size_t ws_bytes, void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
  * Split-KV grouped-query decode attention with a cluster DSMEM merge.
  * [XZY] "CUDA 内核优化与融合", item "Attention内核并行优化"; [NV] "CUDA kernel
  * optimisation and fusion": the work is split along the sequence dimension of
@@ -222,6 +283,60 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
                          int Lcap, const int32_t* seq_lens, float softmax_scale,
                          int cluster_size, uint16_t* out, void* ws, size_t ws_bytes,
                          void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
+ * Split-KV decode attention over an FP8 (e4m3) KV cache.  [TC] and [XZY]
+ * (section "CUDA 内核优化与融合" and the FP8 rationale): FP8 is used for
+ * attention as well as for the GEMMs and MoE; it halves the KV bytes streamed.
+ * Same computation, layout, split, merge and rules as dl_decode_attn, except:
+ *   k_cache, v_cache  e4m3 bytes [B][Hkv][Lcap][d] (OCP E4M3 "e4m3fn"), the
+ *             cache holding k / s_k and v / s_v
+ *   kv_scale  device float[2] = {s_k, s_v}, the per-tensor cache scales (a
+ *             static input: read before the PDL wait)
+ * o = softmax(softmax_scale * q (s_k K)^T) (s_v V).  The tile is converted to
+ * f16 on chip and the products run in f16 with fp32 accumulation (q and the
+ * probabilities are rounded to f16).  Supported: d = 128, (Hq/Hkv)*T <= 32.
+ * The workspace rules are those of dl_decode_attn, sized by
+ * dl_decode_attn_fp8kv_workspace_bytes.
+ * ------------------------------------------------------------------------- */
+dl_status dl_decode_attn_fp8kv(const uint16_t* q, long long q_token_stride, int B, int T, int Hq,
+                               int Hkv, int d, const uint8_t* k_cache, const uint8_t* v_cache,
+                               const float* kv_scale, int Lcap, const int32_t* seq_lens,
+                               float softmax_scale, int cluster_size, uint16_t* out, void* ws,
+                               size_t ws_bytes, void* stream, unsigned flags);
+
+/* Workspace bytes for dl_decode_attn_fp8kv at these shapes (0 for invalid shapes). */
+size_t dl_decode_attn_fp8kv_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Lcap,
+                                            int cluster_size);
+
+/* ---------------------------------------------------------------------------
+ * Greedy speculative verification, on the device.  [XZY] "推测解码" /
+ * "端到端的工作流" (the target verifies the draft tokens of a step in parallel,
+ * keeps those that match the token it would generate itself, and emits its own
+ * token at the first mismatch) and "通过 CUDA Graph 和重叠调度器减少主机端开销"
+ * (the verification stays on the device, inside the step's CUDA graph).
+ *   logits     bf16 [B][T][V]: the target's outputs at the step's T input
+ *              positions (the last accepted token, then the T-1 drafts); finite
+ *   draft_ids  int32 [B][T-1]: the drafts fed at positions 1..T-1 (may be NULL
+ *              when T == 1)
+ *   target_ids int32 [B][T] out: argmax over V of each position (the lowest
+ *              index wins a tie)
+ *   n_accepted int32 [B] out: n = the number of leading drafts with
+ *              draft_ids[b][i] == target_ids[b][i]
+ *   emitted    int32 [B][T] out: target_ids[b][0..n], then -1: the n accepted
+ *              drafts and the target's own next token (n + 1 tokens)
+ *   seq_lens   int32 [B] or NULL: if given, decreased in place by T-1-n, so it
+ *              again counts only the cache entries of accepted tokens (the
+ *              caller's cache held all T inputs of this step)
+ * No workspace; no device-side errors.  Under DL_FLAG_PDL the logits and draft
+ * ids are read after the wait.  seq_lens is written here, so the next call that
+ * reads it (dl_decode_attn) must not immediately follow this one under PDL.
+ * Supported: 1 <= T <= 32, 1 <= B <= 65535, V % 8 == 0; logits 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+dl_status dl_spec_verify_greedy(const uint16_t* logits, int B, int T, int V,
+                                const int32_t* draft_ids, int32_t* target_ids,
+                                int32_t* n_accepted, int32_t* emitted, int32_t* seq_lens,
+                                void* stream, unsigned flags);
 
 /* Workspace bytes for dl_decode_attn at these shapes.  When B*Hkv*cluster_size
  * CTAs would leave the GPU half idle, dl_decode_attn splits each (b, kv head)

@@ -49,8 +49,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
   __shared__ float warp_max[kAqThreads / 32];
   __shared__ float cta_amax;
 
-  // x may be produced by the preceding kernel: wait before reading it, then let
-  // the dependent GEMM start streaming its weights.
+  // x may be produced by the preceding kernel: wait before reading it (through
+  // L2, ld.global.cg), then let the dependent GEMM start streaming its weights.
   pdl_wait();
   pdl_trigger();
 
@@ -71,12 +71,12 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
 #pragma unroll
   for (int j = 0; j < kKeep; ++j) {
     const int i = v0 + threadIdx.x + j * kAqThreads;
-    u[j] = i < v1 ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+    u[j] = i < v1 ? __ldcg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int j = 0; j < kKeep; ++j) m = fmaxf(m, absmax8(u[j]));
   for (int i = v0 + threadIdx.x + kKeep * kAqThreads; i < v1; i += kAqThreads)  // larger inputs
-    m = fmaxf(m, absmax8(__ldg(xv + i)));
+    m = fmaxf(m, absmax8(__ldcg(xv + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const uint16_t* _
       q2[i] = amax > 0.0f ? make_uint2(quant4(u[j].x, u[j].y, inv), quant4(u[j].z, u[j].w, inv)) : make_uint2(0u, 0u);
   }
   for (int i = v0 + threadIdx.x + kKeep * kAqThreads; i < v1; i += kAqThreads) {
-    const uint4 w = __ldg(xv + i);
+    const uint4 w = __ldcg(xv + i);
     q2[i] = amax > 0.0f ? make_uint2(quant4(w.x, w.y, inv), quant4(w.z, w.w, inv)) : make_uint2(0u, 0u);
   }
   if (r == 0 && threadIdx.x == 0) *s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;

@@ -13,24 +13,28 @@
 //    of a thread-block cluster hold S neighbouring chunks.  The G = Hq/Hkv query
 //    heads and the T query tokens share every K/V byte loaded, so K and V are
 //    read exactly once.
-//  * a producer warp moves 64-key tiles of K and V with TMA tensor copies in the
-//    128-byte swizzle (bank-conflict-free ldmatrix), into a ring of stages; it
-//    does not wait for the preceding kernel (the KV cache is static), so under
-//    PDL the ring fills while the QKV GEMM still runs.
-//  * four consumer warps each take 16 keys of a tile and run swapped-AB
-//    tensor-core MMAs (mma.sync m16n8k16, bf16 -> fp32): S^T = K Q^T with the
-//    keys as the M dimension and the R = G*T query rows as N (padded to 8, not
-//    16), then O^T += V^T P^T.  P^T is formed in registers with movmatrix; the
-//    Q^T fragments are read from shared memory, which keeps two CTAs per SM.
-//  * online softmax in the log2 domain; the row max is a 3-step warp shuffle.
-//  * merges: the four warp states merge in shared memory; the S CTA states of
-//    a cluster merge through distributed shared memory (M* = max m_i,
-//    L* = sum l_i 2^(m_i-M*), o = sum o_i 2^(m_i-M*) / L*), each CTA owning
-//    1/S of the outputs.  With P = 1 that is the final result.  With P > 1
-//    (used when B*Hkv*S CTAs would leave the GPU half idle) each cluster
-//    stores its merged state in the workspace and bumps a per-(b, kv head)
+//  * a producer warp moves tiles of 16*W keys of K and V with TMA tensor copies
+//    in the 128-byte swizzle (bank-conflict-free ldmatrix) into a ring of
+//    stages; it does not wait for the preceding kernel (the KV cache is
+//    static), so under PDL the ring fills while the QKV GEMM still runs.
+//  * W consumer warps each take 16 keys of a tile and run swapped-AB
+//    tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation): S^T = K Q^T with
+//    the keys as the M dimension and the R = G*T query rows as N (padded to 8,
+//    not 16), then O^T += V^T P^T.  P^T is formed in registers with movmatrix;
+//    the Q^T fragments are read from shared memory.
+//  * online softmax in the log2 domain with a lazily raised running max; the
+//    row max is a 3-step warp shuffle.
+//  * merges: the W warp states merge in shared memory; each CTA then pushes
+//    its state of every output item (a float4 of o and the row's (m, l)) into
+//    the receive buffer of the CTA of the cluster that owns the item, through
+//    distributed shared memory; after one cluster barrier each owner merges
+//    the S states (M* = max m_i, L* = sum l_i 2^(m_i-M*), o = sum o_i
+//    2^(m_i-M*) / L*).  With P = 1 that is the final result.  With P > 1 (used
+//    when B*Hkv*S CTAs would leave the GPU half idle) each cluster stores its
+//    merged state in the workspace and bumps a per-(b, kv head, owner)
 //    counter; the cluster that arrives last merges the P states the same way
 //    and resets the counter.  Nothing ever waits for another cluster.
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
 #include "dl_device.cuh"
@@ -56,6 +60,7 @@ struct AttnArgs {
   uint32_t* counters;  // [B*Hkv][S], P > 1 only
   float* part_ml;      // [B*Hkv][P][S][R][2] per-owner (m, l)
   float* part_o;       // [B*Hkv][P][R*D/4] float4
+  const float* kv_scale;  // FP8 cache only: device [2] = {s_k, s_v}
   int P;
   int stages;
   int recv_off;        // byte offset of the DSMEM receive buffer
@@ -66,22 +71,32 @@ __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-template <int D, int NT, int W>
+// F8: the KV cache holds e4m3 codes (one byte per element) with per-tensor
+// scales s_k, s_v.  The ring then carries half the bytes; each consumer warp
+// converts its 16 keys of a tile to f16 in a private staging buffer laid out
+// like a bf16 tile (so the ldmatrix paths are shared), frees the ring slot at
+// once, and runs the MMAs in f16 (Q and P are converted to f16 as well).
+template <int D, int NT, int W, bool F8>
 __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                        const __grid_constant__ AttnArgs a) {
+  static_assert(!F8 || D == 128, "the FP8 cache path is built for d = 128");
   constexpr int kAttnConsumers = W;
   constexpr int kAttnThreads = 32 * (W + 1);
   constexpr int kAttnKT = 16 * W;             // keys per pipeline stage
-  constexpr int HALVES = D / 64;              // a swizzled row holds 64 bf16 (128 bytes)
+  constexpr int HALVES = D / 64;              // a swizzled row holds 64 16-bit values (128 bytes)
   constexpr int HALF_BYTES = kAttnKT * 128;   // kAttnKT keys x 128 bytes
-  constexpr int STAGE_BYTES = 2 * HALVES * HALF_BYTES;
+  constexpr int KV_BYTES = F8 ? kAttnKT * D : HALVES * HALF_BYTES;  // one of K, V in a stage
+  constexpr int STAGE_BYTES = 2 * KV_BYTES;
+  constexpr int STG_HALF = 16 * 128;          // f16 staging: 16 keys x 64 d per half
+  constexpr int STG_BYTES = F8 ? 2 * HALVES * STG_HALF : 0;  // per consumer warp: K halves, V halves
   constexpr int KS = D / 16;                  // MMA k-steps over d, and m-tiles of d
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
-  uint2* qs = reinterpret_cast<uint2*>(ring + a.stages * STAGE_BYTES);        // [KS][NT][32]
+  uint8_t* stg_all = ring + a.stages * STAGE_BYTES;                           // [W][STG_BYTES]
+  uint2* qs = reinterpret_cast<uint2*>(stg_all + kAttnConsumers * STG_BYTES);  // [KS][NT][32]
   uint8_t* recv_base = smem + a.recv_off;                                      // DSMEM receive buffer
   uint64_t* bars = reinterpret_cast<uint64_t*>(qs + KS * NT * 32);
   int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages);
@@ -162,10 +177,15 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         const uint32_t fb = full0 + 8u * s;
         mbar_arrive_expect_tx(fb, STAGE_BYTES);
         const int key0 = lo + i * kAttnKT;
+        if (F8) {  // one 128-byte e4m3 row per key: a single box per tensor
+          tma_load_3d(st, &tk, 0, key0, z, fb);
+          tma_load_3d(st + KV_BYTES, &tv, 0, key0, z, fb);
+        } else {
 #pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          tma_load_3d(st + h * HALF_BYTES, &tk, h * 64, key0, z, fb);
-          tma_load_3d(st + (HALVES + h) * HALF_BYTES, &tv, h * 64, key0, z, fb);
+          for (int h = 0; h < HALVES; ++h) {
+            tma_load_3d(st + h * HALF_BYTES, &tk, h * 64, key0, z, fb);
+            tma_load_3d(st + (HALVES + h) * HALF_BYTES, &tv, h * 64, key0, z, fb);
+          }
         }
         issued = i + 1;
       }
@@ -196,10 +216,18 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
             a.q + (static_cast<long long>(b) * a.T + t) * a.q_stride + static_cast<long long>(hq) * D;
         v.x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
         v.y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
+        if (F8) {  // bf16 pairs -> f16 pairs (the f16 MMA needs both operands in f16)
+          v.x = pack_f16x2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u));
+          v.y = pack_f16x2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+        }
       }
       qs[f] = v;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kAttnConsumers) : "memory");
+
+    // F8: the cache holds k / s_k, so the logits take s_k into their scale
+    const float scale_log2 = F8 ? a.scale_log2 * __ldg(a.kv_scale) : a.scale_log2;
+    uint8_t* stg = stg_all + warp * STG_BYTES;
 
     int lim[NT][2];  // last visible key of the rows this thread accumulates
 #pragma unroll
@@ -220,9 +248,45 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
       ok = __all_sync(0xffffffffu, ok);  // the warp-wide MMA path below needs a uniform decision
       const int key_base = lo + i * kAttnKT + warp * 16;
+      bool released = false;
+      if (F8 && ok && key_base < hi) {
+        // e4m3 rows of this warp's 16 keys -> f16 staging in the swizzled bf16-tile
+        // layout; lane = (key r, 64-d half hf), 4 chunks of 16 codes each for K and V.
+        const int r = lane >> 1;
+        const int hf = lane & 1;
+        const int rr = warp * 16 + r;  // row within the stage
+        const uint8_t* kst = ring + s * STAGE_BYTES;
+#pragma unroll
+        for (int t2 = 0; t2 < 2; ++t2) {  // K, then V
+          const uint8_t* src = kst + t2 * KV_BYTES + rr * 128;
+          uint8_t* dst = stg + t2 * HALVES * STG_HALF + hf * STG_HALF + r * 128;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = hf * 4 + c4;  // 16-byte chunk of the 128-byte row: d = 16c .. 16c+15
+            const uint4 u = *reinterpret_cast<const uint4*>(src + ((c ^ (rr & 7)) << 4));
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            uint32_t hv[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2_raw lo2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[e] & 0xFFFFu), __NV_E4M3);
+              const __half2_raw hi2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[e] >> 16), __NV_E4M3);
+              hv[2 * e] = static_cast<uint32_t>(lo2.x) | (static_cast<uint32_t>(lo2.y) << 16);
+              hv[2 * e + 1] = static_cast<uint32_t>(hi2.x) | (static_cast<uint32_t>(hi2.y) << 16);
+            }
+            *reinterpret_cast<uint4*>(dst + (((2 * c4) ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(dst + (((2 * c4 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8u * s);  // the ring slot is free: staging holds the tile
+        released = true;
+      }
       if (ok && key_base < hi) {
-        const uint32_t kbase = smem_u32(ring + s * STAGE_BYTES);
-        const uint32_t vbase = kbase + HALVES * HALF_BYTES;
+        // F8: this warp's staging holds rows 0..15; bf16: the ring holds rows warp*16 ..
+        const int row0 = F8 ? 0 : warp * 16;
+        const int half_bytes = F8 ? STG_HALF : HALF_BYTES;
+        const uint32_t kbase = F8 ? smem_u32(stg) : smem_u32(ring + s * STAGE_BYTES);
+        const uint32_t vbase = kbase + HALVES * half_bytes;
         // ---- S^T[16 keys x 8*NT rows] = K . Q^T ----
         float sc[NT][4];
 #pragma unroll
@@ -231,18 +295,19 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           for (int c = 0; c < 4; ++c) sc[nt][c] = 0.0f;
         {
           const int j = lane >> 3;
-          const int key_l = warp * 16 + (j & 1) * 8 + (lane & 7);
+          const int key_l = row0 + (j & 1) * 8 + (lane & 7);
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             const int half = ks >> 2;
             const int ch = (ks & 3) * 2 + (j >> 1);
-            const uint32_t addr = kbase + half * HALF_BYTES + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
+            const uint32_t addr = kbase + half * half_bytes + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const uint2 qf = qs[(ks * NT + nt) * 32 + lane];
-              mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
+              if (F8) mma_f16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
+              else mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
             }
           }
         }
@@ -255,8 +320,8 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           float p[4];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const float x0 = (kA < hi && kA <= lim[nt][j]) ? sc[nt][j] * a.scale_log2 : -INFINITY;
-            const float x1 = (kB < hi && kB <= lim[nt][j]) ? sc[nt][2 + j] * a.scale_log2 : -INFINITY;
+            const float x0 = (kA < hi && kA <= lim[nt][j]) ? sc[nt][j] * scale_log2 : -INFINITY;
+            const float x1 = (kB < hi && kB <= lim[nt][j]) ? sc[nt][2 + j] * scale_log2 : -INFINITY;
             float mx = fmaxf(x0, x1);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -281,27 +346,30 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
             l_run[nt][j] += p[j] + p[2 + j];
           }
           // P^T as the B operand [k = key][n = row]: transpose each 8x8 block
-          pb[nt][0] = movmatrix_t(pack_bf16x2(p[0], p[1]));
-          pb[nt][1] = movmatrix_t(pack_bf16x2(p[2], p[3]));
+          pb[nt][0] = movmatrix_t(F8 ? pack_f16x2(p[0], p[1]) : pack_bf16x2(p[0], p[1]));
+          pb[nt][1] = movmatrix_t(F8 ? pack_f16x2(p[2], p[3]) : pack_bf16x2(p[2], p[3]));
         }
         // ---- O^T[d x rows] += V^T . P^T ----
         {
           const int j = lane >> 3;
-          const int key_l = warp * 16 + (j >> 1) * 8 + (lane & 7);
+          const int key_l = row0 + (j >> 1) * 8 + (lane & 7);
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
             const int half = mt >> 2;
             const int ch = (mt & 3) * 2 + (j & 1);
-            const uint32_t addr = vbase + half * HALF_BYTES + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
+            const uint32_t addr = vbase + half * half_bytes + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4_t(addr, a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              if (F8) mma_f16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+              else mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8u * s);
+      __syncwarp();  // (F8) every lane is done reading the staging before it is refilled
+      if (!released && lane == 0) mbar_arrive(empty0 + 8u * s);
     }
     // full row sums: add the partial sums of the 8 lanes that share a row
 #pragma unroll
@@ -343,18 +411,17 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   }
   __syncthreads();
 
-  // ---- merge the four warp states and push the CTA state to the slice owners ----
+  // ---- merge the W warp states and push the CTA state to the slice owners ----
   // Outputs are I = R*D/4 float4 items; CTA c of the cluster owns items
-  // [c*Q, (c+1)*Q).  Every CTA stores its state of item i straight into the
-  // receive buffer of the owner of i (remote shared-memory stores, no round
-  // trip), and the (m, l) of each row into every peer; one cluster barrier
-  // later each owner merges the S states of its items locally.
+  // [c*Q, (c+1)*Q).  Every CTA stores its state of item i -- the float4 of o
+  // and the (m, l) of its row -- straight into the receive buffer of the owner
+  // of i (two remote shared-memory stores per item, no round trip); one
+  // cluster barrier later each owner merges the S states of its items locally.
   const int I = R * (D / 4);
   const int Q = (I + S - 1) / S;
-  float4* rv_o = reinterpret_cast<float4*>(recv_base);     // [S][Q]
-  float* rv_m = reinterpret_cast<float*>(rv_o + S * Q);   // [S][R]
-  float* rv_l = rv_m + S * R;                             // [S][R]
-  const uint32_t rv_o_l = smem_u32(rv_o), rv_m_l = smem_u32(rv_m), rv_l_l = smem_u32(rv_l);
+  float4* rv_o = reinterpret_cast<float4*>(recv_base);      // [S][Q]
+  float2* rv_ml = reinterpret_cast<float2*>(rv_o + S * Q);  // [S][Q] (m, l)
+  const uint32_t rv_o_l = smem_u32(rv_o), rv_ml_l = smem_u32(rv_ml);
   for (int it = threadIdx.x; it < I; it += kAttnThreads) {
     const int rho = it / (D / 4);
     const int c4 = it - rho * (D / 4);
@@ -378,17 +445,14 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
     }
     const int owner = it / Q;
-    dsmem_st_f32x4(dsmem_addr(rv_o_l + 16u * (rank * Q + (it - owner * Q)), owner), acc);
-    if (c4 == 0) {
-      for (int p = 0; p < S; ++p) {
-        dsmem_st_f32(dsmem_addr(rv_m_l + 4u * (rank * R + rho), p), M);
-        dsmem_st_f32(dsmem_addr(rv_l_l + 4u * (rank * R + rho), p), lsum);
-      }
-    }
+    const uint32_t slot_i = static_cast<uint32_t>(rank * Q + (it - owner * Q));
+    dsmem_st_f32x4(dsmem_addr(rv_o_l + 16u * slot_i, owner), acc);
+    dsmem_st_f32x2(dsmem_addr(rv_ml_l + 8u * slot_i, owner), M, lsum);
   }
   cluster_sync();  // every state of my items has landed in my receive buffer
 
   // ---- merge the S CTA states of my items ----
+  const float out_scale = F8 ? __ldg(a.kv_scale + 1) : 1.0f;  // F8: the cache holds v / s_v
   const long long head = static_cast<long long>(b) * a.Hkv + hk;
   const long long slot = head * a.P + split;
   const int my0 = rank * Q;
@@ -399,13 +463,13 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     const int c4 = it - rho * (D / 4);
     float M = -INFINITY;
     for (int p = 0; p < S; ++p)
-      if (rv_l[p * R + rho] > 0.0f) M = fmaxf(M, rv_m[p * R + rho]);
+      if (rv_ml[p * Q + k].y > 0.0f) M = fmaxf(M, rv_ml[p * Q + k].x);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.0f;
     for (int p = 0; p < S; ++p) {
-      const float lp = rv_l[p * R + rho];
+      const float lp = rv_ml[p * Q + k].y;
       if (lp > 0.0f) {
-        const float f = ex2(rv_m[p * R + rho] - M);
+        const float f = ex2(rv_ml[p * Q + k].x - M);
         const float4 v = rv_o[p * Q + k];
         acc.x += v.x * f;
         acc.y += v.y * f;
@@ -415,7 +479,7 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
     }
     if (a.P == 1) {
-      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      const float inv = lsum > 0.0f ? out_scale / lsum : 0.0f;
       const int t = rho / a.G;
       const int hq = hk * a.G + rho % a.G;
       uint16_t* dst = a.out + ((static_cast<long long>(b) * a.T + t) * a.Hq + hq) * D + c4 * 4;
@@ -474,7 +538,7 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
             lsum += lq * f;
           }
         }
-        const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+        const float inv = lsum > 0.0f ? out_scale / lsum : 0.0f;
         const int t = rho / a.G;
         const int hq = hk * a.G + rho % a.G;
         uint16_t* dst = a.out + ((static_cast<long long>(b) * a.T + t) * a.Hq + hq) * D + c4 * 4;
@@ -503,16 +567,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-static bool encode_kv_map(CUtensorMap* m, const uint16_t* base, int d, int Lcap, int BH, int kt) {
+// K or V cache [BH][Lcap][d] as a 3-D tensor map with 128-byte rows per box:
+// bf16 elements in boxes of 64 (two boxes per key for d = 128), or e4m3 bytes
+// in one box of d = 128.
+static bool encode_kv_map(CUtensorMap* m, const void* base, int d, int Lcap, int BH, int kt, bool fp8) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
+  const cuuint64_t esz = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Lcap), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(Lcap) * d * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kt), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz, static_cast<cuuint64_t>(Lcap) * d * esz};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(kt), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Workspace of dl_decode_attn with P clusters per (b, kv head) of S CTAs: the
@@ -533,49 +601,49 @@ struct AttnPlan {
   int stages, smem, recv_off;
 };
 
-template <int D, int NT, int W>
+template <int D, int NT, int W, bool F8>
 static AttnPlan attn_plan(int R, int S) {
-  constexpr int STAGE_BYTES = 2 * (D / 64) * (16 * W) * 128;
+  constexpr int STAGE_BYTES = F8 ? 2 * (16 * W) * D : 2 * (D / 64) * (16 * W) * 128;
+  constexpr int STG = F8 ? W * 2 * (D / 64) * 16 * 128 : 0;  // f16 staging of all consumer warps
   const int merge_bytes = (W * R * D + 2 * W * R) * 4;
   const int I = R * (D / 4);
   const int Q = (I + S - 1) / S;
-  const int recv_bytes = S * Q * 16 + 2 * S * R * 4;
+  const int recv_bytes = S * Q * (16 + 8);
   const int qs_bytes = (D / 16) * NT * 32 * 8;
-  auto smem_for = [&](int st) { return 1024 + st * STAGE_BYTES + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16; };
+  auto smem_for = [&](int st) {
+    return 1024 + st * STAGE_BYTES + STG + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16;
+  };
   int stages = W == 4 ? (D == 128 ? 3 : 6) : (D == 128 ? 3 : 6);
   if (W == 8 || 2 * (smem_for(stages) + 1024) > 233472) {
     stages = 6;
     while (stages > 2 && smem_for(stages) > 232448) --stages;
   }
-  while (stages * STAGE_BYTES < merge_bytes) ++stages;
+  while (stages * STAGE_BYTES + STG < merge_bytes) ++stages;  // the merge reuses ring + staging
   AttnPlan pl;
   pl.stages = stages;
   pl.smem = smem_for(stages);
-  pl.recv_off = ((stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
+  pl.recv_off = ((stages * STAGE_BYTES + STG + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
   return pl;
 }
 
-template <int D, int NT, int W>
+template <int D, int NT, int W, bool F8>
 static cudaError_t attn_configure(const AttnPlan& pl, int S) {
-  auto kern = decode_attn_kernel<D, NT, W>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
-  if (e == cudaSuccess && S > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  return e;
+  return ensure_kernel_attrs(reinterpret_cast<const void*>(decode_attn_kernel<D, NT, W, F8>), pl.smem, S > 8);
 }
 
 // Clusters of S CTAs of this kernel that can be resident on the GPU at once.
-template <int D, int NT, int W>
+template <int D, int NT, int W, bool F8>
 static int attn_max_clusters_t(int R, int S) {
-  const AttnPlan pl = attn_plan<D, NT, W>(R, S);
+  const AttnPlan pl = attn_plan<D, NT, W, F8>(R, S);
   const int per_sm = 233472 / (pl.smem + 1024) >= 2 ? 2 : 1;
   int fallback = (sm_count() * per_sm) / S;
-  if (attn_configure<D, NT, W>(pl, S) != cudaSuccess) {
+  if (attn_configure<D, NT, W, F8>(pl, S) != cudaSuccess) {
     (void)cudaGetLastError();
     return fallback;
   }
   Launch L(dim3(S, 1, 1), dim3(32 * (W + 1)), static_cast<size_t>(pl.smem), nullptr, static_cast<unsigned>(S), false);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, NT, W>, &L.cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_attn_kernel<D, NT, W, F8>, &L.cfg) != cudaSuccess || n < 1) {
     (void)cudaGetLastError();
     return fallback;
   }
@@ -584,74 +652,101 @@ static int attn_max_clusters_t(int R, int S) {
 
 static int attn_warps(int S) { return S >= 16 ? 4 : 8; }
 
-template <int W>
+template <int W, bool F8>
 static int attn_max_clusters_w(int d, int R, int S) {
   const int NT = (R + 7) / 8;
-  if (d == 128) {
+  if (F8 || d == 128) {
     switch (NT) {
-      case 1: return attn_max_clusters_t<128, 1, W>(R, S);
-      case 2: return attn_max_clusters_t<128, 2, W>(R, S);
-      case 3: return attn_max_clusters_t<128, 3, W>(R, S);
-      default: return attn_max_clusters_t<128, 4, W>(R, S);
+      case 1: return attn_max_clusters_t<128, 1, W, F8>(R, S);
+      case 2: return attn_max_clusters_t<128, 2, W, F8>(R, S);
+      case 3: return attn_max_clusters_t<128, 3, W, F8>(R, S);
+      default: return attn_max_clusters_t<128, 4, W, F8>(R, S);
     }
   }
   switch (NT) {
-    case 1: return attn_max_clusters_t<64, 1, W>(R, S);
-    case 2: return attn_max_clusters_t<64, 2, W>(R, S);
-    case 3: return attn_max_clusters_t<64, 3, W>(R, S);
-    default: return attn_max_clusters_t<64, 4, W>(R, S);
+    case 1: return attn_max_clusters_t<64, 1, W, false>(R, S);
+    case 2: return attn_max_clusters_t<64, 2, W, false>(R, S);
+    case 3: return attn_max_clusters_t<64, 3, W, false>(R, S);
+    default: return attn_max_clusters_t<64, 4, W, false>(R, S);
   }
 }
 
-static int attn_max_clusters(int d, int R, int S) {
-  return attn_warps(S) == 8 ? attn_max_clusters_w<8>(d, R, S) : attn_max_clusters_w<4>(d, R, S);
+struct AttnShapeKey {
+  int d, R, S;
+  bool fp8;
+};
+
+static int attn_max_clusters_query(const void* ctx) {
+  const AttnShapeKey& k = *static_cast<const AttnShapeKey*>(ctx);
+  if (k.fp8)
+    return attn_warps(k.S) == 8 ? attn_max_clusters_w<8, true>(k.d, k.R, k.S)
+                                : attn_max_clusters_w<4, true>(k.d, k.R, k.S);
+  return attn_warps(k.S) == 8 ? attn_max_clusters_w<8, false>(k.d, k.R, k.S)
+                              : attn_max_clusters_w<4, false>(k.d, k.R, k.S);
+}
+
+// The occupancy query costs a runtime round trip: asked once per device and shape.
+static int attn_max_clusters(int d, int R, int S, bool fp8) {
+  const AttnShapeKey k{d, R, S, fp8};
+  const unsigned long long key = (1ull << 60) | (static_cast<unsigned long long>(fp8) << 48) |
+                                 (static_cast<unsigned long long>(d) << 32) |
+                                 (static_cast<unsigned long long>(R) << 16) | static_cast<unsigned long long>(S);
+  return memo_int(key, attn_max_clusters_query, &k);
 }
 
 // Clusters per (b, kv head).  Splitting a head over P clusters costs a merge
 // through the workspace (~2-3 us), so it is used only when each CTA would
 // otherwise stream long chunks (>= 2048 keys), with >= 1024 keys per CTA
 // left, and never beyond the clusters that can be resident at once.
-int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R) {
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R, bool fp8) {
   const long long keys_per_cta = Lcap / cluster;
   if (keys_per_cta < 2048) return 1;
   const long long heads = static_cast<long long>(B) * Hkv;
-  const long long resident = attn_max_clusters(d, R, cluster);
+  const long long resident = attn_max_clusters(d, R, cluster, fp8);
   long long P = resident / heads;
   if (P > keys_per_cta / 1024) P = keys_per_cta / 1024;
   if (P > kAttnMaxSplits) P = kAttnMaxSplits;
   return P < 1 ? 1 : static_cast<int>(P);
 }
 
-template <int D, int NT, int W>
+template <int D, int NT, int W, bool F8>
 static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                                  const AttnLaunch& p, cudaStream_t s) {
-  const AttnPlan pl = attn_plan<D, NT, W>(a.R, p.cluster);
+  const AttnPlan pl = attn_plan<D, NT, W, F8>(a.R, p.cluster);
   AttnArgs args = a;
   args.stages = pl.stages;
   args.recv_off = pl.recv_off;
-  cudaError_t e = attn_configure<D, NT, W>(pl, p.cluster);
+  cudaError_t e = attn_configure<D, NT, W, F8>(pl, p.cluster);
   if (e != cudaSuccess) return e;
   Launch L(dim3(p.cluster, p.Hkv, p.B * a.P), dim3(32 * (W + 1)), static_cast<size_t>(pl.smem), s,
            static_cast<unsigned>(p.cluster), p.pdl);
-  return cudaLaunchKernelEx(&L.cfg, decode_attn_kernel<D, NT, W>, tk, tv, args);
+  return cudaLaunchKernelEx(&L.cfg, decode_attn_kernel<D, NT, W, F8>, tk, tv, args);
 }
 
 template <int W>
 static cudaError_t launch_attn_w(const CUtensorMap& tk, const CUtensorMap& tv, const AttnArgs& a,
                                  const AttnLaunch& p, cudaStream_t s, int NT) {
-  if (p.d == 128) {
+  if (p.fp8) {
+    if (p.d != 128) return cudaErrorInvalidValue;
     switch (NT) {
-      case 1: return launch_attn_t<128, 1, W>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<128, 2, W>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<128, 3, W>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<128, 4, W>(tk, tv, a, p, s);
+      case 1: return launch_attn_t<128, 1, W, true>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<128, 2, W, true>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<128, 3, W, true>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<128, 4, W, true>(tk, tv, a, p, s);
+    }
+  } else if (p.d == 128) {
+    switch (NT) {
+      case 1: return launch_attn_t<128, 1, W, false>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<128, 2, W, false>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<128, 3, W, false>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<128, 4, W, false>(tk, tv, a, p, s);
     }
   } else if (p.d == 64) {
     switch (NT) {
-      case 1: return launch_attn_t<64, 1, W>(tk, tv, a, p, s);
-      case 2: return launch_attn_t<64, 2, W>(tk, tv, a, p, s);
-      case 3: return launch_attn_t<64, 3, W>(tk, tv, a, p, s);
-      case 4: return launch_attn_t<64, 4, W>(tk, tv, a, p, s);
+      case 1: return launch_attn_t<64, 1, W, false>(tk, tv, a, p, s);
+      case 2: return launch_attn_t<64, 2, W, false>(tk, tv, a, p, s);
+      case 3: return launch_attn_t<64, 3, W, false>(tk, tv, a, p, s);
+      case 4: return launch_attn_t<64, 4, W, false>(tk, tv, a, p, s);
     }
   }
   return cudaErrorInvalidValue;
@@ -661,8 +756,8 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   const int W = attn_warps(p.cluster);
   const int kt = 16 * W;  // keys per stage of the chosen variant
   CUtensorMap tk, tv;
-  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt) ||
-      !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt))
+  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8) ||
+      !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = p.q;
@@ -681,12 +776,13 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   a.stages = 3;
   a.debug = p.debug ? 1 : 0;
   // clusters per (b, kv head): forced, else automatic; then as many as the workspace holds
-  int P = p.splits > 0 ? p.splits : attn_auto_splits(p.B, p.Hkv, p.cluster, p.Lcap, p.d, a.R);
+  int P = p.splits > 0 ? p.splits : attn_auto_splits(p.B, p.Hkv, p.cluster, p.Lcap, p.d, a.R, p.fp8);
   while (P > 1 && attn_ws_bytes(p.B, p.Hkv, a.R, p.d, P, p.cluster) > p.ws_bytes) --P;
   if (static_cast<long long>(p.B) * P > 65535) P = 1;
   a.P = P;
   a.counters = nullptr;
   a.part_ml = a.part_o = nullptr;
+  a.kv_scale = p.kv_scale;
   if (P > 1) {
     const size_t heads = static_cast<size_t>(p.B) * p.Hkv;
     uint8_t* base = reinterpret_cast<uint8_t*>(p.status) + kWsHeader;

@@ -37,6 +37,16 @@ struct Launch {
 };
 
 int sm_count();  // SMs of the current device (cached per device)
+int current_device();
+
+// Raises the dynamic shared-memory limit of a kernel (and allows non-portable
+// cluster sizes) on the current device only when a launch needs more than was
+// set before: launches after the first cost no runtime call.
+cudaError_t ensure_kernel_attrs(const void* func, int smem_bytes, bool nonportable_cluster);
+
+// Memoised per (device, key): returns the cached value, or computes it with
+// fn(), stores it and returns it.  Thread-safe.
+int memo_int(unsigned long long key, int (*fn)(const void*), const void* ctx);
 
 // Workspace layout (see dl.h).
 constexpr size_t kWsHeader = 256;
@@ -47,6 +57,11 @@ inline uint8_t* ws_xq(void* ws) { return static_cast<uint8_t*>(ws) + kWsHeader; 
 // ---- kernels' host launchers (return a CUDA error code) ----
 cudaError_t launch_act_quant(const uint16_t* x, int M, int K, uint8_t* xq, float* s_x,
                              cudaStream_t s, bool pdl);
+cudaError_t launch_add_rmsnorm_quant(const uint16_t* x, const uint16_t* r, uint16_t* h_out, const uint16_t* gamma,
+                                     int M, int K, float eps, uint8_t* xq, float* s_x, cudaStream_t s, bool pdl);
+cudaError_t launch_spec_verify(const uint16_t* logits, int B, int T, int V, const int32_t* draft,
+                               int32_t* target_ids, int32_t* n_accepted, int32_t* emitted, int32_t* seq_lens,
+                               cudaStream_t s, bool pdl);
 cudaError_t launch_pack(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
                         cudaStream_t s);
 
@@ -77,8 +92,10 @@ struct AttnLaunch {
   const uint16_t* q;
   long long q_stride;
   int B, T, Hq, Hkv, d, Lcap;
-  const uint16_t* k;
-  const uint16_t* v;
+  const void* k;              // bf16 [B][Hkv][Lcap][d], or e4m3 bytes when fp8
+  const void* v;
+  bool fp8;                   // e4m3 cache with kv_scale = device {s_k, s_v}
+  const float* kv_scale;
   const int32_t* seq_lens;
   float scale;
   int cluster;
@@ -91,6 +108,6 @@ struct AttnLaunch {
 };
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t s);
 size_t attn_ws_bytes(int B, int Hkv, int R, int d, int P, int S);
-int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R);
+int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R, bool fp8);
 
 }  // namespace dl

@@ -175,7 +175,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   __syncthreads();
   const int n_tok = misc->n_tok;
   const int expert = misc->expert;
-  if (n_tok == 0) return;  // unused expert slot: every CTA of the cluster leaves here
+  if (n_tok == 0) {  // unused expert slot: every CTA of the cluster leaves here
+    // One early leaver still waits for the predecessor, so that this grid never
+    // completes before it even when no slot is used (completion stays ordered
+    // along the PDL chain).
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == gridDim.z - 1) pdl_wait();
+    return;
+  }
   const int npad = (n_tok + 7) & ~7;
   const bool routed = a.expert_ids != nullptr;
 
@@ -298,6 +304,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     if (a.x != nullptr) {
       // Fused quantiser (A1): amax over the whole [M][K] input, then this CTA's
       // K slice straight into the B operand.  Same arithmetic as act_quant.cu.
+      // x (like x_q and s_x below) may be written by the preceding kernel while
+      // this one already runs, so it is read through L2 (ld.global.cg), never
+      // through the read-only path.
       const uint4* xv = reinterpret_cast<const uint4*>(a.x);
       const int nv = (a.M * a.K) >> 3;
       // This thread's first kKeep chunks of the CTA's K slice are loaded into
@@ -315,8 +324,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
           const int rem = c - row * per_row;
           const uint4* src =
               xv + ((static_cast<long long>(row) * a.K + (kb0 + (rem >> 3)) * 128 + (rem & 7) * 16) >> 3);
-          keep[2 * j] = __ldg(src);
-          keep[2 * j + 1] = __ldg(src + 1);
+          keep[2 * j] = __ldcg(src);
+          keep[2 * j + 1] = __ldcg(src + 1);
         }
       }
       // amax over all of x: 16 independent 16-byte loads in flight per thread per
@@ -328,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
           const int i = base + 64 * j;
-          u[j] = i < nv ? __ldg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
+          u[j] = i < nv ? __ldcg(xv + i) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) m = fmaxf(m, absmax8(u[j]));
@@ -359,8 +368,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
               }
           } else {
             const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + kbl) * 128 + ch * 16) >> 3);
-            u0 = __ldg(src);
-            u1 = __ldg(src + 1);
+            u0 = __ldcg(src);
+            u1 = __ldcg(src + 1);
           }
           v = make_uint4(quant4(u0.x, u0.y, inv), quant4(u0.z, u0.w, inv), quant4(u1.x, u1.y, inv),
                          quant4(u1.z, u1.w, inv));
@@ -374,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       fence_async_smem();
       mbar_arrive(xready);
     } else {
-    if (t == 0) misc->sx = __ldg(a.s_x);
+    if (t == 0) misc->sx = __ldcg(a.s_x);
     // Stream the e4m3 activations of each k-block into the B ring, one slot
     // ahead of the MMAs that read it; every 16-byte chunk is an independent
     // async copy, so a whole k-block is in flight at once.
@@ -476,15 +485,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   {
     const int row = warp * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    for (int c0 = 0; c0 < SUBS * npad; c0 += 8) {
-      uint32_t r[8];
-      tmem_ld_x8(lane_base + static_cast<uint32_t>(c0), r);
+    const int ncols = SUBS * npad;
+    for (int c0 = 0; c0 < ncols; c0 += 32) {  // up to four 8-column loads in flight per wait
+      uint32_t r[4][8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (c0 + 8 * q < ncols) tmem_ld_x8(lane_base + static_cast<uint32_t>(c0 + 8 * q), r[q]);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = c0 + j;
-        const int m = col % npad;
-        if (m < n_tok) part[col * 128 + row] = __uint_as_float(r[j]);
+      for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = c0 + 8 * q + j;
+          const int m = col % npad;
+          if (col < ncols && m < n_tok) part[col * 128 + row] = __uint_as_float(r[q][j]);
+        }
       }
     }
   }
@@ -496,40 +511,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   const int rows = 128 * (rank + 1) / S - r0;
   const int items = rows * n_tok;
   const uint32_t part_base = smem_u32(part);
-  for (int it = threadIdx.x; it < items; it += kGemmThreads) {
-    const int m = it / rows;
-    const int row = r0 + (it - m * rows);
-    const int tok = routed ? misc->tokens[m] : m;
-    const uint32_t off_g = part_base + static_cast<uint32_t>((m * 128 + row) * 4);
-    float gv[8], uv[8];
+  // kPullBatch items per thread per round: all their peer loads are issued
+  // before the first sum, so a round costs one DSMEM round trip, not one per item.
+  constexpr int kPullBatch = 4;
+  for (int it0 = threadIdx.x; it0 < items; it0 += kGemmThreads * kPullBatch) {
+    float gv[kPullBatch][8], uv[kPullBatch][8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {  // issue every peer load before the first add
-      if (p < S) {
-        gv[p] = dsmem_ld_f32(dsmem_addr(off_g, p));
-        uv[p] = kSwiglu ? dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p)) : 0.0f;
+    for (int q = 0; q < kPullBatch; ++q) {
+      const int it = it0 + q * kGemmThreads;
+      const int m = it / rows;
+      const int row = r0 + (it - m * rows);
+      const uint32_t off_g = part_base + static_cast<uint32_t>((m * 128 + row) * 4);
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        gv[q][p] = 0.0f;
+        uv[q][p] = 0.0f;
+        if (it < items && p < S) {
+          gv[q][p] = dsmem_ld_f32(dsmem_addr(off_g, p));
+          if (kSwiglu) uv[q][p] = dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p));
+        }
       }
     }
-    float g = 0.0f;
-    float u = 0.0f;
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      if (p < S) {
-        g += gv[p];
-        u += uv[p];
+    for (int q = 0; q < kPullBatch; ++q) {
+      const int it = it0 + q * kGemmThreads;
+      if (it >= items) continue;
+      const int m = it / rows;
+      const int row = r0 + (it - m * rows);
+      const int tok = routed ? misc->tokens[m] : m;
+      float g = 0.0f;
+      float u = 0.0f;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {  // peers summed in rank order
+        g += gv[q][p];
+        u += uv[q][p];
       }
-    }
-    if (kSwiglu) {
-      const float yg = g * scale;
-      const float yu = u * scale;
-      const float o = yg / (1.0f + expf(-yg)) * yu;
-      const __nv_bfloat16 b = __float2bfloat16_rn(o);
-      a.out[static_cast<long long>(tok) * a.ldo + tile * 128 + row] = *reinterpret_cast<const uint16_t*>(&b);
-    } else {
-      const int col = tile * 128 + row;
-      float y = g * scale;
-      if (col < a.q_cols) y *= a.q_scale;
-      const __nv_bfloat16 b = __float2bfloat16_rn(y);
-      a.out[static_cast<long long>(tok) * a.ldo + col] = *reinterpret_cast<const uint16_t*>(&b);
+      if (kSwiglu) {
+        const float yg = g * scale;
+        const float yu = u * scale;
+        const float o = yg / (1.0f + expf(-yg)) * yu;
+        const __nv_bfloat16 b = __float2bfloat16_rn(o);
+        a.out[static_cast<long long>(tok) * a.ldo + tile * 128 + row] = *reinterpret_cast<const uint16_t*>(&b);
+      } else {
+        const int col = tile * 128 + row;
+        float y = g * scale;
+        if (col < a.q_cols) y *= a.q_scale;
+        const __nv_bfloat16 b = __float2bfloat16_rn(y);
+        a.out[static_cast<long long>(tok) * a.ldo + col] = *reinterpret_cast<const uint16_t*>(&b);
+      }
     }
   }
   tc_fence_before();
@@ -621,11 +650,11 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
            static_cast<unsigned>(S), g.pdl);
   cudaError_t e;
   if (g.swiglu) {
-    e = cudaFuncSetAttribute(gemm_e4m3_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = ensure_kernel_attrs(reinterpret_cast<const void*>(gemm_e4m3_kernel<true>), smem, false);
     if (e != cudaSuccess) return e;
     return cudaLaunchKernelEx(&L.cfg, gemm_e4m3_kernel<true>, a);
   }
-  e = cudaFuncSetAttribute(gemm_e4m3_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = ensure_kernel_attrs(reinterpret_cast<const void*>(gemm_e4m3_kernel<false>), smem, false);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&L.cfg, gemm_e4m3_kernel<false>, a);
 }

@@ -1,0 +1,235 @@
+// norm_quant.cu -- residual add + RMSNorm + Quantize: the producer of an FP8
+// GEMM input, as one kernel.
+//
+// [XZY] "CUDA 内核优化与融合", item "运算融合", and [NV] "CUDA kernel
+// optimisation and fusion" fuse (AllReduce +) RMSNorm + Quantize into one
+// kernel ahead of the FP8 GEMM.  On one GPU the AllReduce is absent; the
+// residual add of the pre-norm block takes its place:
+//   h = bf16_rne(x + r)                         (the residual stream, bf16)
+//   y = (h * rsqrt(mean(h^2) + eps)) * gamma     (fp32, per token row)
+//   amax = max|y| over the whole [M][K] tensor, inv = 448/amax, s_x = amax/448
+//   x_q = e4m3_rn_satfinite(y * inv)
+// x_q and s_x land in a GEMM workspace, whose GEMM then runs with
+// DL_FLAG_XQ_READY and skips its own quantisation.
+//
+// One thread-block cluster of C <= 8 CTAs covers the tensor.  Each CTA owns R
+// consecutive token rows and 16/R warps per row; a row's h stays in registers
+// from the load to the quantisation, so x and r are read from memory once.
+// Row sums of squares are reduced in a fixed order (deterministic), the
+// tensor amax across the cluster through distributed shared memory.
+#include <cuda_fp8.h>
+
+#include "dl_device.cuh"
+#include "dl_internal.h"
+
+namespace dl {
+
+constexpr int kNqThreads = 512;
+constexpr int kNqWarps = kNqThreads / 32;
+constexpr int kNqKeep = 10;  // 16-byte vectors of h per thread held in registers
+
+struct NormQuantArgs {
+  const uint16_t* x;
+  const uint16_t* r;      // may be null
+  uint16_t* h_out;        // may be null
+  const uint16_t* gamma;  // [K]
+  uint8_t* xq;            // [M][K]
+  float* s_x;
+  int M, K;
+  int R;                  // rows per CTA (power of two, <= 16)
+  float eps;
+};
+
+__device__ __forceinline__ float nq_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float nq_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// bf16 round-to-nearest-even of the fp32 sum of two bf16 pairs, packed.  The
+// fp32 sum of two bf16 values is exact unless their exponents differ by more
+// than 16, and then the smaller operand is below half an ulp of the result's
+// bf16 grid, so one further rounding to bf16 equals rounding the exact sum.
+__device__ __forceinline__ uint32_t add2_bf16(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 s = __floats2bfloat162_rn(__fadd_rn(nq_lo(a), nq_lo(b)), __fadd_rn(nq_hi(a), nq_hi(b)));
+  return *reinterpret_cast<const uint32_t*>(&s);
+}
+
+__device__ __forceinline__ uint4 add8_bf16(uint4 a, uint4 b) {
+  return make_uint4(add2_bf16(a.x, b.x), add2_bf16(a.y, b.y), add2_bf16(a.z, b.z), add2_bf16(a.w, b.w));
+}
+
+__device__ __forceinline__ float sumsq8(uint4 u) {
+  float s = 0.0f;
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s = __fmaf_rn(nq_lo(w[i]), nq_lo(w[i]), s);
+    s = __fmaf_rn(nq_hi(w[i]), nq_hi(w[i]), s);
+  }
+  return s;
+}
+
+// y = (h * rs) * gamma for 8 values; returns max |y| and fills y.
+__device__ __forceinline__ float norm8(uint4 h, uint4 g, float rs, float* y) {
+  const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+  const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    y[2 * i] = __fmul_rn(__fmul_rn(nq_lo(hw[i]), rs), nq_lo(gw[i]));
+    y[2 * i + 1] = __fmul_rn(__fmul_rn(nq_hi(hw[i]), rs), nq_hi(gw[i]));
+    m = fmaxf(m, fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1])));
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint2 quant8(const float* y, float inv) {
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(y[2 * i], inv), __fmul_rn(y[2 * i + 1], inv)), __NV_SATFINITE, __NV_E4M3);
+    q[i] = static_cast<uint32_t>(p);
+  }
+  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+}
+
+// h of vector v again, beyond the register set: from h_out when this thread
+// stored it there (whatever h_out aliases), else recomputed from x and r.
+__device__ __forceinline__ uint4 reload_h(const uint4* xv, const uint4* rv, const uint4* hv, int v) {
+  if (hv != nullptr) return __ldcg(hv + v);
+  const uint4 u = __ldcg(xv + v);
+  return rv != nullptr ? add8_bf16(u, __ldcg(rv + v)) : u;
+}
+
+// Launched as one cluster of gridDim.x CTAs.
+__global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __grid_constant__ NormQuantArgs a) {
+  __shared__ float red[kNqWarps];
+  __shared__ float cta_amax;
+
+  // x and r may be produced by the preceding kernel: wait before reading them,
+  // then let the dependent GEMM start streaming its weights.
+  pdl_wait();
+  pdl_trigger();
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = gridDim.x;
+  const int crank = static_cast<int>(cluster_rank());
+  const int WR = kNqWarps / a.R;          // warps per row
+  const int TPR = WR * 32;                // threads per row
+  const int rr = warp / WR;
+  const int tr = (warp - rr * WR) * 32 + lane;
+  const int row = crank * a.R + rr;
+  const bool live = row < a.M;
+  const int VR = a.K >> 3;                // 16-byte vectors per row
+  const long long rbase = static_cast<long long>(row) * VR;
+  const uint4* xv = reinterpret_cast<const uint4*>(a.x) + rbase;
+  const uint4* rv = a.r != nullptr ? reinterpret_cast<const uint4*>(a.r) + rbase : nullptr;
+  uint4* hv = a.h_out != nullptr ? reinterpret_cast<uint4*>(a.h_out) + rbase : nullptr;
+  const uint4* gv = reinterpret_cast<const uint4*>(a.gamma);
+
+  // ---- h = x (+ r), kept in registers; row sum of squares -------------------
+  uint4 h[kNqKeep];
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kNqKeep; ++j) {
+    const int v = tr + j * TPR;
+    h[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (live && v < VR) {
+      h[j] = __ldcg(xv + v);
+      if (rv != nullptr) h[j] = add8_bf16(h[j], __ldcg(rv + v));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kNqKeep; ++j) {
+    const int v = tr + j * TPR;
+    if (live && v < VR) {
+      if (hv != nullptr) hv[v] = h[j];
+      ss += sumsq8(h[j]);
+    }
+  }
+  for (int v = tr + kNqKeep * TPR; live && v < VR; v += TPR) {  // rows longer than the register set
+    uint4 u = __ldcg(xv + v);
+    if (rv != nullptr) u = add8_bf16(u, __ldcg(rv + v));
+    if (hv != nullptr) hv[v] = u;
+    ss += sumsq8(u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int w = 0; w < WR; ++w) tot += red[rr * WR + w];  // fixed order: deterministic
+  const float rs = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, static_cast<float>(a.K)), a.eps));
+  __syncthreads();  // red[] is reused below
+
+  // ---- amax of y over the tensor ----------------------------------------------
+  float m = 0.0f;
+  float y[8];
+#pragma unroll
+  for (int j = 0; j < kNqKeep; ++j) {
+    const int v = tr + j * TPR;
+    if (live && v < VR) m = fmaxf(m, norm8(h[j], __ldg(gv + v), rs, y));
+  }
+  for (int v = tr + kNqKeep * TPR; live && v < VR; v += TPR) {
+    const uint4 u = reload_h(xv, rv, hv, v);
+    m = fmaxf(m, norm8(u, __ldg(gv + v), rs, y));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float w = threadIdx.x < kNqWarps ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+    if (threadIdx.x == 0) cta_amax = w;
+  }
+  cluster_sync();  // every CTA's maximum is visible cluster-wide
+  float amax = 0.0f;
+  const uint32_t local = smem_u32(&cta_amax);
+  for (int p = 0; p < C; ++p) amax = fmaxf(amax, dsmem_ld_f32(dsmem_addr(local, p)));
+
+  // ---- quantise from registers ------------------------------------------------
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
+  uint2* q2 = reinterpret_cast<uint2*>(a.xq) + rbase;
+#pragma unroll
+  for (int j = 0; j < kNqKeep; ++j) {
+    const int v = tr + j * TPR;
+    if (live && v < VR) {
+      norm8(h[j], __ldg(gv + v), rs, y);
+      q2[v] = amax > 0.0f ? quant8(y, inv) : make_uint2(0u, 0u);
+    }
+  }
+  for (int v = tr + kNqKeep * TPR; live && v < VR; v += TPR) {
+    const uint4 u = reload_h(xv, rv, hv, v);
+    norm8(u, __ldg(gv + v), rs, y);
+    q2[v] = amax > 0.0f ? quant8(y, inv) : make_uint2(0u, 0u);
+  }
+  if (crank == 0 && threadIdx.x == 0) *a.s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+
+  cluster_sync();  // peers have finished reading cta_amax before this CTA exits
+}
+
+cudaError_t launch_add_rmsnorm_quant(const uint16_t* x, const uint16_t* r, uint16_t* h_out, const uint16_t* gamma,
+                                     int M, int K, float eps, uint8_t* xq, float* s_x, cudaStream_t s, bool pdl) {
+  // rows per CTA: the smallest power of two that fits M rows in <= 8 CTAs
+  int R = 1;
+  while (R < 16 && (M + R - 1) / R > 8) R <<= 1;
+  const int C = (M + R - 1) / R;
+  if (C > 8) return cudaErrorInvalidValue;
+  NormQuantArgs a;
+  a.x = x;
+  a.r = r;
+  a.h_out = h_out;
+  a.gamma = gamma;
+  a.xq = xq;
+  a.s_x = s_x;
+  a.M = M;
+  a.K = K;
+  a.R = R;
+  a.eps = eps;
+  Launch L(dim3(C), dim3(kNqThreads), 0, s, static_cast<unsigned>(C), pdl);
+  return cudaLaunchKernelEx(&L.cfg, add_rmsnorm_quant_kernel, a);
+}
+
+}  // namespace dl

@@ -25,6 +25,9 @@ import numpy as np
 import torch
 
 E4M3_MAX = 448.0
+# Vocabulary of the verification workloads: the size of Llama 4 Maverick's
+# tokenizer (the pages do not state it; public model configuration).
+VOCAB = 202048
 
 
 @dataclasses.dataclass(frozen=True)
@@ -42,11 +45,21 @@ class Workload:
     L: int              # KV length (fixed) or 0 when drawn per sequence
     Lcap: int           # KV cache capacity per sequence
     experts: int = 0    # MoE experts (0 = dense)
-    cluster: int = 8    # attention split-KV cluster size
+    cluster: int = 8    # attention split-KV cluster size (the measured best for the shape)
 
     @property
     def n_qkv(self) -> int:
         return (self.Hq + 2 * self.Hkv) * self.d
+
+    @property
+    def k_o(self) -> int:
+        """Attention output projection: reduction length Hq*d, output rows K."""
+        return self.Hq * self.d
+
+    @property
+    def k_fc2(self) -> int:
+        """FC2 down projection: reduction length F = N2/2, output rows K."""
+        return self.N2 // 2
 
 
 WORKLOADS = {
@@ -55,9 +68,9 @@ WORKLOADS = {
     "layer_b1": Workload("layer_b1", 1, K=5120, M=1, N2=16384, Hq=40, Hkv=8, d=128, B=1, T=1,
                          L=4096, Lcap=4096, cluster=8),
     "verify4": Workload("verify4", 2, K=5120, M=4, N2=16384, Hq=40, Hkv=8, d=128, B=1, T=4,
-                        L=32768, Lcap=32768, cluster=8),
+                        L=32768, Lcap=32768, cluster=4),
     "batch16x4": Workload("batch16x4", 3, K=5120, M=64, N2=16384, Hq=40, Hkv=8, d=128, B=16,
-                          T=4, L=0, Lcap=16384, cluster=8),
+                          T=4, L=0, Lcap=16384, cluster=4),
     "moe64": Workload("moe64", 4, K=5120, M=64, N2=16384, Hq=40, Hkv=8, d=128, B=0, T=0, L=0,
                       Lcap=0, experts=128),
 }
@@ -114,6 +127,11 @@ def expert_ids_for(wl: Workload, g: np.random.Generator) -> np.ndarray:
     return g.integers(0, wl.experts, size=wl.M).astype(np.int32)
 
 
+def rmsnorm_gain(g: np.random.Generator, K: int) -> np.ndarray:
+    """A synthetic RMSNorm gain: bf16 of 1 + 0.1 N(0, 1)."""
+    return bf16_bits(np.float32(1.0) + g.standard_normal(size=K, dtype=np.float32) * np.float32(0.1))
+
+
 def dense_layer_inputs(wl: Workload, with_weights: bool = True, with_kv: bool = True):
     """Host arrays for one dense decode layer of workload ``wl``.
 
@@ -133,4 +151,24 @@ def dense_layer_inputs(wl: Workload, with_weights: bool = True, with_kv: bool = 
         out["seq_lens"] = seq_lens_for(wl, g)
         out["k_cache"] = bf16_normal(g, (wl.B, wl.Hkv, wl.Lcap, wl.d))
         out["v_cache"] = bf16_normal(g, (wl.B, wl.Hkv, wl.Lcap, wl.d))
+    return out
+
+
+def full_layer_inputs(wl: Workload):
+    """Host arrays for the whole pre-norm layer of workload ``wl``: x (the
+    previous layer's output) and h (the residual stream) [M, K] bf16; weights
+    w_qkv, w_o [K, Hq*d], w13, w2 [K, F] e4m3 with their scales; RMSNorm gains
+    g1, g2 [K] bf16; the KV caches, seq_lens and q_scale."""
+    g = rng(1000 + wl.seed)
+    out = {"x": bf16_normal(g, (wl.M, wl.K)), "h": bf16_normal(g, (wl.M, wl.K)),
+           "q_scale": np.float32(1.0 / math.sqrt(wl.d))}
+    out["w_qkv"], out["s_qkv"] = e4m3_weight(g, wl.n_qkv, wl.K)
+    out["w_o"], out["s_o"] = e4m3_weight(g, wl.K, wl.k_o)
+    out["w13"], out["s13"] = e4m3_weight(g, wl.N2, wl.K)
+    out["w2"], out["s2"] = e4m3_weight(g, wl.K, wl.k_fc2)
+    out["g1"] = rmsnorm_gain(g, wl.K)
+    out["g2"] = rmsnorm_gain(g, wl.K)
+    out["seq_lens"] = seq_lens_for(wl, g)
+    out["k_cache"] = bf16_normal(g, (wl.B, wl.Hkv, wl.Lcap, wl.d))
+    out["v_cache"] = bf16_normal(g, (wl.B, wl.Hkv, wl.Lcap, wl.d))
     return out

@@ -28,6 +28,7 @@ DL_ERR_DEVICE_ARG = 7
 
 DL_FLAG_PDL = 1
 DL_FLAG_DEBUG_TIMEOUT = 2
+DL_FLAG_XQ_READY = 4
 DL_FLAG_SPLIT_SHIFT = 8
 DL_PACK_PLAIN = 0
 DL_PACK_SWIGLU = 1
@@ -47,8 +48,14 @@ _SIGNATURES = {
     "dl_fc13_swiglu_static_ws": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _P, _U]),
     "dl_fc_qkv_scale": (_I, [_P, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P, _SZ, _P, _U]),
     "dl_moe_fc13_swiglu_grouped": (_I, [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
+    "dl_gemm_e4m3": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
+    "dl_moe_gemm_grouped": (_I, [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
+    "dl_add_rmsnorm_quant": (_I, [_P, _P, _P, _P, _I, _I, _F, _P, _SZ, _P, _U]),
+    "dl_spec_verify_greedy": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _U]),
     "dl_decode_attn": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
     "dl_decode_attn_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "dl_decode_attn_fp8kv": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
+    "dl_decode_attn_fp8kv_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "dl_read_status": (_I, [_P, _P]),
     "dl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -138,11 +145,45 @@ def dl_moe_fc13_swiglu_grouped(x, T, K, expert_ids, E, w_packed, w_scales, N2, o
                                             _stream(stream), flags)
 
 
+def dl_gemm_e4m3(x, M, K, w_packed, w_scale, N, out, ws, ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
+    return lib().dl_gemm_e4m3(_ptr(x), M, K, _ptr(w_packed), _ptr(w_scale), N, _ptr(out), _ptr(ws),
+                              _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_moe_gemm_grouped(x, T, K, expert_ids, E, w_packed, w_scales, N, out, ws, ws_bytes=None, stream=None,
+                        flags=DL_FLAG_PDL) -> int:
+    return lib().dl_moe_gemm_grouped(_ptr(x), T, K, _ptr(expert_ids), E, _ptr(w_packed), _ptr(w_scales), N,
+                                     _ptr(out), _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_add_rmsnorm_quant(x, residual, h_out, gamma, M, K, eps, ws, ws_bytes=None, stream=None,
+                         flags=DL_FLAG_PDL) -> int:
+    return lib().dl_add_rmsnorm_quant(_ptr(x), _ptr(residual), _ptr(h_out), _ptr(gamma), M, K, float(eps),
+                                      _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_spec_verify_greedy(logits, B, T, V, draft_ids, target_ids, n_accepted, emitted, seq_lens=None, stream=None,
+                          flags=DL_FLAG_PDL) -> int:
+    return lib().dl_spec_verify_greedy(_ptr(logits), B, T, V, _ptr(draft_ids), _ptr(target_ids), _ptr(n_accepted),
+                                       _ptr(emitted), _ptr(seq_lens), _stream(stream), flags)
+
+
 def dl_decode_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, Lcap, seq_lens, softmax_scale,
                    cluster_size, out, ws, ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
     return lib().dl_decode_attn(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(v_cache),
                                 Lcap, _ptr(seq_lens), float(softmax_scale), cluster_size, _ptr(out), _ptr(ws),
                                 _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_decode_attn_fp8kv(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, kv_scale, Lcap, seq_lens,
+                         softmax_scale, cluster_size, out, ws, ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
+    return lib().dl_decode_attn_fp8kv(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(kv_scale), Lcap, _ptr(seq_lens), float(softmax_scale), cluster_size,
+                                      _ptr(out), _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_decode_attn_fp8kv_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size) -> int:
+    return int(lib().dl_decode_attn_fp8kv_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size))
 
 
 def dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size) -> int:

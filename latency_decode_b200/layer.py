@@ -50,8 +50,11 @@ class DecodeLayer:
         self.Lcap_hint = None
         self.ws_attn = None
         self.qkv = torch.empty((M, self.N_qkv), dtype=torch.int16, device=self.device)
-        self.attn_out = torch.empty((B, T, Hq, d), dtype=torch.int16, device=self.device)
-        self.ffn_out = torch.empty((M, self.N2 // 2), dtype=torch.int16, device=self.device)
+        # both results in one buffer, so a caller can fetch them with one copy
+        n_attn = B * T * Hq * d
+        self.out_buf = torch.empty(n_attn + M * (self.N2 // 2), dtype=torch.int16, device=self.device)
+        self.attn_out = self.out_buf[:n_attn].view(B, T, Hq, d)
+        self.ffn_out = self.out_buf[n_attn:].view(M, self.N2 // 2)
 
     @property
     def weight_bytes(self) -> int:
@@ -76,5 +79,92 @@ class DecodeLayer:
 
     def read_status(self, stream=None) -> None:
         for ws in (self.ws_qkv, self.ws_attn, self.ws_13):
+            if ws is not None:
+                dl.check(dl.dl_read_status(ws, stream))
+
+
+class FullDecodeLayer:
+    """The whole pre-norm decode layer of a dense model on one GPU:
+
+        h  <- x + h;  x1 = RMSNorm(h) * g1 -> e4m3          (dl_add_rmsnorm_quant)
+        qkv = FC_QKV(x1) with the Q columns scaled          (dl_fc_qkv_scale, x_q from the norm)
+        o   = attention(q, K cache, V cache)                (dl_decode_attn, q read in place)
+        a   = O_proj(o)                                     (dl_gemm_e4m3)
+        h  <- a + h;  x2 = RMSNorm(h) * g2 -> e4m3          (dl_add_rmsnorm_quant)
+        f   = SwiGLU(FC13(x2))                              (dl_fc13_swiglu, x_q from the norm)
+        y   = FC2(f)                                        (dl_gemm_e4m3)
+
+    ``y`` is the layer's output and ``h`` its residual stream; the next layer's
+    first step adds them.  Seven kernels (eight or nine when an input is too
+    large for a GEMM to quantise itself), chained with PDL on one stream.
+    Every step runs in libdl.so; this class only holds buffers."""
+
+    def __init__(self, w_qkv, s_qkv, w_o, s_o, w13, s13, w2, s2, g1, g2, *, Hq, Hkv, d, q_scale, M, B, T,
+                 eps: float = 1e-5, cluster: int = 8, device="cuda"):
+        """Weights: canonical e4m3 bytes (uint8, on device) in nn.Linear [N, K] order:
+        w_qkv [(Hq+2Hkv)d, D], w_o [D, Hq d], w13 [2F, D], w2 [D, F].  g1, g2:
+        bf16 bits [D] (int16, on device)."""
+        assert M == B * T
+        self.device = torch.device(device)
+        self.Hq, self.Hkv, self.d, self.M, self.B, self.T = Hq, Hkv, d, M, B, T
+        self.cluster, self.eps, self.q_scale = cluster, float(eps), float(q_scale)
+        self.N_qkv, self.D = w_qkv.shape
+        self.N2 = w13.shape[0]
+        self.F = self.N2 // 2
+        assert w_o.shape == (self.D, Hq * d) and w2.shape == (self.D, self.F)
+        self.wp = {}
+        for name, w, kind in (("qkv", w_qkv, dl.DL_PACK_PLAIN), ("o", w_o, dl.DL_PACK_PLAIN),
+                              ("13", w13, dl.DL_PACK_SWIGLU), ("2", w2, dl.DL_PACK_PLAIN)):
+            p = torch.empty_like(w)
+            dl.check(dl.dl_pack_fp8_weight(w, p, w.shape[0], w.shape[1], kind))
+            self.wp[name] = p
+        self.s = {k: _scale_tensor(v, self.device) for k, v in (("qkv", s_qkv), ("o", s_o), ("13", s13),
+                                                                 ("2", s2))}
+        self.g1, self.g2 = g1, g2
+
+        def ws(K):
+            return torch.zeros(dl.dl_workspace_bytes(M, K), dtype=torch.uint8, device=self.device)
+
+        self.ws_qkv, self.ws_o, self.ws_13, self.ws_2 = ws(self.D), ws(Hq * d), ws(self.D), ws(self.F)
+        self.ws_attn = None
+        self.Lcap_hint = None
+        self.qkv = torch.empty((M, self.N_qkv), dtype=torch.int16, device=self.device)
+        self.attn_out = torch.empty((M, Hq * d), dtype=torch.int16, device=self.device)
+        self.a = torch.empty((M, self.D), dtype=torch.int16, device=self.device)
+        self.f = torch.empty((M, self.F), dtype=torch.int16, device=self.device)
+        self.y = torch.empty((M, self.D), dtype=torch.int16, device=self.device)
+
+    @property
+    def weight_bytes(self) -> int:
+        return sum(int(p.numel()) for p in self.wp.values())
+
+    def step(self, x, h, k_cache, v_cache, seq_lens, stream=None, flags: int = dl.DL_FLAG_PDL) -> None:
+        """x: the previous layer's output, h: the residual stream (updated in
+        place), both bf16 bits [M, D]; caches [B, Hkv, Lcap, d]; seq_lens int32
+        [B].  The output lands in self.y."""
+        M, D = self.M, self.D
+        Lcap = k_cache.shape[2]
+        if self.ws_attn is None or self.Lcap_hint != Lcap:
+            n = dl.dl_decode_attn_workspace_bytes(self.B, self.T, self.Hq, self.Hkv, self.d, Lcap, self.cluster)
+            self.ws_attn = torch.zeros(n, dtype=torch.uint8, device=self.device)
+            self.Lcap_hint = Lcap
+        ready = flags | dl.DL_FLAG_XQ_READY
+        dl.check(dl.dl_add_rmsnorm_quant(x, h, h, self.g1, M, D, self.eps, self.ws_qkv, stream=stream, flags=flags))
+        dl.check(dl.dl_fc_qkv_scale(None, M, D, self.wp["qkv"], self.s["qkv"], self.Hq, self.Hkv, self.d,
+                                    self.q_scale, self.qkv, self.ws_qkv, stream=stream, flags=ready))
+        dl.check(dl.dl_decode_attn(self.qkv, self.N_qkv, self.B, self.T, self.Hq, self.Hkv, self.d, k_cache,
+                                   v_cache, Lcap, seq_lens, 1.0, self.cluster, self.attn_out, self.ws_attn,
+                                   stream=stream, flags=flags))
+        dl.check(dl.dl_gemm_e4m3(self.attn_out, M, self.Hq * self.d, self.wp["o"], self.s["o"], D, self.a,
+                                 self.ws_o, stream=stream, flags=flags))
+        dl.check(dl.dl_add_rmsnorm_quant(self.a, h, h, self.g2, M, D, self.eps, self.ws_13, stream=stream,
+                                         flags=flags))
+        dl.check(dl.dl_fc13_swiglu(None, M, D, self.wp["13"], self.s["13"], self.N2, self.f, self.ws_13,
+                                   stream=stream, flags=ready))
+        dl.check(dl.dl_gemm_e4m3(self.f, M, self.F, self.wp["2"], self.s["2"], D, self.y, self.ws_2,
+                                 stream=stream, flags=flags))
+
+    def read_status(self, stream=None) -> None:
+        for ws in (self.ws_qkv, self.ws_attn, self.ws_o, self.ws_13, self.ws_2):
             if ws is not None:
                 dl.check(dl.dl_read_status(ws, stream))

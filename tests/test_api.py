@@ -174,3 +174,80 @@ def test_pack_reference_is_a_permutation_with_the_stated_layout():
         blk = 2 * (t * KB + kb)
         assert p[blk * 16384 + intra] == w[j, k]
         assert p[(blk + 1) * 16384 + intra] == w[F + j, k]
+
+
+def test_plain_and_grouped_projection_argument_errors():
+    base = dict(x=FAKE, M=1, K=512, w_packed=FAKE, w_scale=FAKE, N=256, out=FAKE, ws=FAKE, ws_bytes=1 << 20,
+                stream=0, flags=0)
+    assert dl.dl_gemm_e4m3(**{**base, "x": None}) == dl.DL_ERR_INVALID_ARG  # x needed without XQ_READY
+    assert dl.dl_gemm_e4m3(**{**base, "N": 64}) == dl.DL_ERR_INVALID_ARG
+    assert dl.dl_gemm_e4m3(**{**base, "N": 320}) == dl.DL_ERR_UNSUPPORTED
+    assert dl.dl_gemm_e4m3(**{**base, "M": 64, "K": 8320}) == dl.DL_ERR_UNSUPPORTED  # M*K > 64*8192
+    assert dl.dl_gemm_e4m3(**{**base, "out": FAKE + 2}) == dl.DL_ERR_ALIGNMENT
+    assert dl.dl_gemm_e4m3(**{**base, "ws_bytes": 256 + 511}) == dl.DL_ERR_WORKSPACE
+    assert dl.dl_gemm_e4m3(**{**base, "flags": 9 << dl.DL_FLAG_SPLIT_SHIFT}) == dl.DL_ERR_INVALID_ARG
+    m = dict(x=FAKE, T=4, K=512, expert_ids=FAKE, E=8, w_packed=FAKE, w_scales=FAKE, N=128, out=FAKE, ws=FAKE,
+             ws_bytes=1 << 20, stream=0, flags=0)
+    assert dl.dl_moe_gemm_grouped(**{**m, "N": 192}) == dl.DL_ERR_UNSUPPORTED
+    assert dl.dl_moe_gemm_grouped(**{**m, "expert_ids": None}) == dl.DL_ERR_INVALID_ARG
+    assert dl.dl_moe_gemm_grouped(**{**m, "E": 1025}) == dl.DL_ERR_UNSUPPORTED
+    assert dl.dl_moe_gemm_grouped(**{**m, "T": 0}) == dl.DL_ERR_INVALID_ARG
+    # the plain grouped entry accepts N % 128 where the SwiGLU one needs N % 256
+    assert dl.dl_moe_fc13_swiglu_grouped(**{**{k: v for k, v in m.items() if k != "N"}, "N2": 128}) \
+        == dl.DL_ERR_INVALID_ARG
+
+
+def _norm(**kw):
+    a = dict(x=FAKE, residual=FAKE + (1 << 24), h_out=FAKE + (2 << 24), gamma=FAKE + (3 << 24), M=4, K=5120,
+             eps=1e-5, ws=FAKE + (4 << 24), ws_bytes=1 << 20, stream=0, flags=0)
+    a.update(kw)
+    return dl.dl_add_rmsnorm_quant(**a)
+
+
+def test_rmsnorm_quant_argument_errors():
+    assert _norm(x=None) == dl.DL_ERR_INVALID_ARG
+    assert _norm(gamma=None) == dl.DL_ERR_INVALID_ARG
+    assert _norm(eps=0.0) == dl.DL_ERR_INVALID_ARG
+    assert _norm(eps=-1.0) == dl.DL_ERR_INVALID_ARG
+    assert _norm(eps=float("nan")) == dl.DL_ERR_INVALID_ARG
+    assert _norm(eps=float("inf")) == dl.DL_ERR_INVALID_ARG
+    assert _norm(M=0) == dl.DL_ERR_INVALID_ARG
+    assert _norm(K=5000) == dl.DL_ERR_UNSUPPORTED
+    assert _norm(M=65) == dl.DL_ERR_UNSUPPORTED
+    assert _norm(M=64, K=8320) == dl.DL_ERR_UNSUPPORTED
+    assert _norm(gamma=FAKE + (3 << 24) + 2) == dl.DL_ERR_ALIGNMENT
+    assert _norm(residual=FAKE + (1 << 24) + 8) == dl.DL_ERR_ALIGNMENT
+    assert _norm(h_out=FAKE + 4096) == dl.DL_ERR_INVALID_ARG  # partial overlap with x
+    assert _norm(h_out=FAKE + (1 << 24) - 4096) == dl.DL_ERR_INVALID_ARG  # partial overlap with residual
+    assert _norm(ws_bytes=256 + 4 * 5120 - 1) == dl.DL_ERR_WORKSPACE
+    assert _norm(ws=None) == dl.DL_ERR_WORKSPACE
+
+
+def test_spec_verify_argument_errors():
+    base = dict(logits=FAKE, B=2, T=4, V=1024, draft_ids=FAKE, target_ids=FAKE, n_accepted=FAKE, emitted=FAKE,
+                seq_lens=None, stream=0, flags=0)
+    f = dl.dl_spec_verify_greedy
+    assert f(**{**base, "logits": None}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**base, "draft_ids": None}) == dl.DL_ERR_INVALID_ARG  # T > 1 needs drafts
+    assert f(**{**base, "T": 0}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**base, "V": 4}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**base, "T": 33}) == dl.DL_ERR_UNSUPPORTED
+    assert f(**{**base, "V": 1001}) == dl.DL_ERR_UNSUPPORTED
+    assert f(**{**base, "B": 70000}) == dl.DL_ERR_UNSUPPORTED
+    assert f(**{**base, "logits": FAKE + 8}) == dl.DL_ERR_ALIGNMENT
+    assert f(**{**base, "seq_lens": FAKE + 2}) == dl.DL_ERR_ALIGNMENT
+    assert f(**{**base, "emitted": None}) == dl.DL_ERR_INVALID_ARG
+
+
+def test_fp8kv_attention_argument_errors():
+    a = dict(q=FAKE, q_token_stride=1024, B=1, T=1, Hq=8, Hkv=2, d=128, k_cache=FAKE, v_cache=FAKE, kv_scale=FAKE,
+             Lcap=256, seq_lens=FAKE, softmax_scale=0.125, cluster_size=8, out=FAKE, ws=FAKE, ws_bytes=256,
+             stream=0, flags=0)
+    f = dl.dl_decode_attn_fp8kv
+    assert f(**{**a, "kv_scale": None}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**a, "d": 64, "q_token_stride": 512}) == dl.DL_ERR_UNSUPPORTED  # the e4m3 path is d = 128 only
+    assert f(**{**a, "k_cache": FAKE + 8}) == dl.DL_ERR_ALIGNMENT
+    assert f(**{**a, "kv_scale": FAKE + 2}) == dl.DL_ERR_ALIGNMENT
+    assert f(**{**a, "cluster_size": 3}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**a, "ws_bytes": 255}) == dl.DL_ERR_WORKSPACE
+    assert dl.dl_decode_attn_fp8kv_workspace_bytes(1, 1, 8, 2, 64, 256, 8) == 0
