@@ -61,6 +61,7 @@ struct AttnArgs {
   float* part_ml;      // [B*Hkv][P][S][R][2] per-owner (m, l)
   float* part_o;       // [B*Hkv][P][R*D/4] float4
   const float* kv_scale;  // FP8 cache only: device [2] = {s_k, s_v}
+  int lpt;             // 1: grid z visits the sequences longest first
   int P;
   int stages;
   int recv_off;        // byte offset of the DSMEM receive buffer
@@ -110,9 +111,31 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   const int S = gridDim.x;
   const int rank = static_cast<int>(cluster_rank());
   const int hk = blockIdx.y;
-  const int b = blockIdx.z / a.P;
-  const int split = blockIdx.z - b * a.P;
+  const int zb = blockIdx.z / a.P;  // dispatch slot of the sequence
+  const int split = blockIdx.z - zb * a.P;
   const long long budget = a.debug ? kWaitBudgetDebug : kWaitBudget;
+
+  // Longest-first order: CTAs are dispatched in grid order, so when the grid
+  // runs in several waves, mapping slot zb to the zb-th longest sequence (ties
+  // by index) makes the hardware's in-order dispatch a longest-processing-time
+  // schedule.  seq_lens is a static input, read before the PDL wait.
+  __shared__ int lpt_seq;
+  int b = zb;
+  if (a.lpt) {
+    for (int j = threadIdx.x; j < a.B; j += blockDim.x) {
+      int Lj = __ldg(a.seq_lens + j);
+      Lj = (Lj < a.T || Lj > a.Lcap) ? 0 : Lj;
+      int rank_j = 0;
+      for (int i = 0; i < a.B; ++i) {
+        int Li = __ldg(a.seq_lens + i);
+        Li = (Li < a.T || Li > a.Lcap) ? 0 : Li;
+        rank_j += (Li > Lj || (Li == Lj && i < j)) ? 1 : 0;
+      }
+      if (rank_j == zb) lpt_seq = j;
+    }
+    __syncthreads();
+    b = lpt_seq;
+  }
 
   // ---- this CTA's key chunk ----
   int L = __ldg(a.seq_lens + b);
@@ -783,6 +806,7 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   a.counters = nullptr;
   a.part_ml = a.part_o = nullptr;
   a.kv_scale = p.kv_scale;
+  a.lpt = (p.B > 1 && p.B <= 128) ? 1 : 0;  // the in-kernel ranking is O(B^2 / threads)
   if (P > 1) {
     const size_t heads = static_cast<size_t>(p.B) * p.Hkv;
     uint8_t* base = reinterpret_cast<uint8_t*>(p.status) + kWsHeader;
