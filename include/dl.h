@@ -348,6 +348,22 @@ dl_status dl_spec_verify_greedy(const uint16_t* logits, int B, int T, int V,
 size_t dl_decode_attn_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int Lcap,
                                       int cluster_size);
 
+/* ---------------------------------------------------------------------------
+ * A copy as a kernel, so that a step which fetches its activations from the
+ * host (or returns its results there) stays one PDL chain.  [XZY]
+ * "程序化依赖启动（PDL）" and [NV] "Programmatic Dependent Launch": the next
+ * kernel's independent preamble (a GEMM's weight stream) overlaps the one
+ * before it; a copy node of a CUDA graph is not a kernel and would break that.
+ *   src, dst  device memory, or pinned host memory from cudaHostAlloc (which
+ *             kernels address directly under unified addressing); 16-byte
+ *             aligned, not overlapping
+ *   bytes     a multiple of 16 (0 launches nothing)
+ * With DL_FLAG_PDL the kernel waits for its predecessor before it reads src or
+ * writes dst.  Host memory written this way is visible to the host once the
+ * stream has been synchronised.
+ * ------------------------------------------------------------------------- */
+dl_status dl_copy(const void* src, void* dst, size_t bytes, void* stream, unsigned flags);
+
 /* Synchronises `stream`, reads the status word of `ws`, clears it, and returns
  * DL_OK, DL_ERR_TIMEOUT or DL_ERR_DEVICE_ARG (timeout takes precedence). */
 dl_status dl_read_status(void* ws, void* stream);

@@ -636,7 +636,10 @@ static AttnPlan attn_plan(int R, int S) {
   auto smem_for = [&](int st) {
     return 1024 + st * STAGE_BYTES + STG + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16;
   };
-  int stages = W == 4 ? (D == 128 ? 3 : 6) : (D == 128 ? 3 : 6);
+  int stages = D == 128 ? 3 : 6;
+  // W = 4 is chosen to put two CTAs on each SM: give up ring depth (down to
+  // two stages) before that
+  while (W == 4 && stages > 2 && 2 * (smem_for(stages) + 1024) > 233472) --stages;
   if (W == 8 || 2 * (smem_for(stages) + 1024) > 233472) {
     stages = 6;
     while (stages > 2 && smem_for(stages) > 232448) --stages;
@@ -673,7 +676,11 @@ static int attn_max_clusters_t(int R, int S) {
   return n;
 }
 
-static int attn_warps(int S) { return S >= 16 ? 4 : 8; }
+// Consumer warps per CTA.  W = 8 (one CTA per SM) when the grid fits in one
+// wave; W = 4 (two CTAs per SM, each overlapping the other's start-up and
+// merge) for 16-CTA clusters and for grids of more CTAs than SMs, where a CTA's
+// fixed costs would otherwise repeat once per wave (batch16x4: 118 -> 97 us).
+static int attn_warps(int S, long long ctas) { return (S >= 16 || ctas > sm_count()) ? 4 : 8; }
 
 template <int W, bool F8>
 static int attn_max_clusters_w(int d, int R, int S) {
@@ -695,23 +702,22 @@ static int attn_max_clusters_w(int d, int R, int S) {
 }
 
 struct AttnShapeKey {
-  int d, R, S;
+  int d, R, S, W;
   bool fp8;
 };
 
 static int attn_max_clusters_query(const void* ctx) {
   const AttnShapeKey& k = *static_cast<const AttnShapeKey*>(ctx);
   if (k.fp8)
-    return attn_warps(k.S) == 8 ? attn_max_clusters_w<8, true>(k.d, k.R, k.S)
-                                : attn_max_clusters_w<4, true>(k.d, k.R, k.S);
-  return attn_warps(k.S) == 8 ? attn_max_clusters_w<8, false>(k.d, k.R, k.S)
-                              : attn_max_clusters_w<4, false>(k.d, k.R, k.S);
+    return k.W == 8 ? attn_max_clusters_w<8, true>(k.d, k.R, k.S) : attn_max_clusters_w<4, true>(k.d, k.R, k.S);
+  return k.W == 8 ? attn_max_clusters_w<8, false>(k.d, k.R, k.S) : attn_max_clusters_w<4, false>(k.d, k.R, k.S);
 }
 
 // The occupancy query costs a runtime round trip: asked once per device and shape.
-static int attn_max_clusters(int d, int R, int S, bool fp8) {
-  const AttnShapeKey k{d, R, S, fp8};
-  const unsigned long long key = (1ull << 60) | (static_cast<unsigned long long>(fp8) << 48) |
+static int attn_max_clusters(int d, int R, int S, bool fp8, int W) {
+  const AttnShapeKey k{d, R, S, W, fp8};
+  const unsigned long long key = (1ull << 60) | (static_cast<unsigned long long>(W) << 52) |
+                                 (static_cast<unsigned long long>(fp8) << 48) |
                                  (static_cast<unsigned long long>(d) << 32) |
                                  (static_cast<unsigned long long>(R) << 16) | static_cast<unsigned long long>(S);
   return memo_int(key, attn_max_clusters_query, &k);
@@ -725,7 +731,7 @@ int attn_auto_splits(int B, int Hkv, int cluster, int Lcap, int d, int R, bool f
   const long long keys_per_cta = Lcap / cluster;
   if (keys_per_cta < 2048) return 1;
   const long long heads = static_cast<long long>(B) * Hkv;
-  const long long resident = attn_max_clusters(d, R, cluster, fp8);
+  const long long resident = attn_max_clusters(d, R, cluster, fp8, attn_warps(cluster, heads * cluster));
   long long P = resident / heads;
   if (P > keys_per_cta / 1024) P = keys_per_cta / 1024;
   if (P > kAttnMaxSplits) P = kAttnMaxSplits;
@@ -776,7 +782,7 @@ static cudaError_t launch_attn_w(const CUtensorMap& tk, const CUtensorMap& tv, c
 }
 
 cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
-  const int W = attn_warps(p.cluster);
+  const int W = attn_warps(p.cluster, static_cast<long long>(p.B) * p.Hkv * p.cluster);
   const int kt = 16 * W;  // keys per stage of the chosen variant
   CUtensorMap tk, tv;
   if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8) ||

@@ -368,6 +368,14 @@ dl_status dl_decode_attn_fp8kv(const uint16_t* q, long long q_token_stride, int 
                   softmax_scale, cluster_size, out, ws, ws_bytes, stream, flags);
 }
 
+dl_status dl_copy(const void* src, void* dst, size_t bytes, void* stream, unsigned flags) {
+  if (src == nullptr || dst == nullptr) return DL_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(dst, 16) || bytes % 16 != 0) return DL_ERR_ALIGNMENT;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(src), b0 = reinterpret_cast<uintptr_t>(dst);
+  if (bytes > 0 && a0 < b0 + bytes && b0 < a0 + bytes) return DL_ERR_INVALID_ARG;  // overlap
+  return cuda_status(dl::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream), (flags & DL_FLAG_PDL) != 0));
+}
+
 dl_status dl_read_status(void* ws, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return DL_ERR_WORKSPACE;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);

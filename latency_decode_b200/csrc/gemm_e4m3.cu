@@ -384,16 +384,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       mbar_arrive(xready);
     } else {
     if (t == 0) misc->sx = __ldcg(a.s_x);
-    // Stream the e4m3 activations of each k-block into the B ring, one slot
-    // ahead of the MMAs that read it; every 16-byte chunk is an independent
-    // async copy, so a whole k-block is in flight at once.
-    for (int kbl = 0; kbl < nkb; ++kbl) {
-      const int bslot = kbl % kBStages;
-      if (kbl >= kBStages &&
-          !mbar_wait(bempty0 + 8u * bslot, static_cast<uint32_t>((kbl / kBStages) - 1) & 1u, budget, abort_flag)) {
+    // Stream the e4m3 activations of each k-block into the B ring with 16-byte
+    // async copies, one commit group per k-block, kBStages-1 k-blocks in
+    // flight: a block is published (bfull) as soon as its own group has landed,
+    // so the L2 latency of one block overlaps the copies of the next ones.
+    auto issue_kb = [&](int kb) -> bool {
+      const int bslot = kb % kBStages;
+      if (kb >= kBStages &&
+          !mbar_wait(bempty0 + 8u * bslot, static_cast<uint32_t>((kb / kBStages) - 1) & 1u, budget, abort_flag)) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
-        break;
+        return false;
       }
       uint8_t* blk = bsm + bslot * npad * 128;
       for (int c = t; c < npad * 8; c += 64) {
@@ -402,15 +403,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
         uint8_t* dst = blk + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
         if (row < n_tok) {
           const int tok = routed ? misc->tokens[row] : row;
-          cp_async_16(smem_u32(dst), a.xq + static_cast<long long>(tok) * a.K + (kb0 + kbl) * 128 + ch * 16);
+          cp_async_16(smem_u32(dst), a.xq + static_cast<long long>(tok) * a.K + (kb0 + kb) * 128 + ch * 16);
         } else {
           *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      cp_async_wait_all();
-      fence_async_smem();
-      mbar_arrive(bfull0 + 8u * bslot);
+      return true;
+    };
+    int committed = 0;  // commit groups so far, one per k-block issued (empty ones at the tail)
+    bool alive = true;
+    for (int kb = 0; kb < nkb && kb < kBStages - 1; ++kb) {
+      alive = alive && issue_kb(kb);
+      cp_async_commit();
+      ++committed;
     }
+    for (int kbl = 0; kbl < nkb && alive; ++kbl) {
+      // publish k-block kbl as soon as its own group has landed ...
+      cp_async_wait_pending(committed - (kbl + 1));
+      fence_async_smem();
+      mbar_arrive(bfull0 + 8u * (kbl % kBStages));
+      // ... then refill the slot k-block kbl-1 used, once its MMAs are done
+      // (waiting for them before the publish would chain the MMAs to this warp)
+      const int kb_next = kbl + kBStages - 1;
+      if (kb_next < nkb) alive = issue_kb(kb_next);
+      cp_async_commit();
+      ++committed;
+    }
+    cp_async_wait_pending(0);  // nothing in flight when the stager moves on
     }
   }
 

@@ -56,6 +56,7 @@ _SIGNATURES = {
     "dl_decode_attn_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "dl_decode_attn_fp8kv": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
     "dl_decode_attn_fp8kv_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "dl_copy": (_I, [_P, _P, _SZ, _P, _U]),
     "dl_read_status": (_I, [_P, _P]),
     "dl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -188,6 +189,10 @@ def dl_decode_attn_fp8kv_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size) -
 
 def dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size) -> int:
     return int(lib().dl_decode_attn_workspace_bytes(B, T, Hq, Hkv, d, Lcap, cluster_size))
+
+
+def dl_copy(src, dst, nbytes, stream=None, flags=DL_FLAG_PDL) -> int:
+    return lib().dl_copy(_ptr(src), _ptr(dst), int(nbytes), _stream(stream), flags)
 
 
 def dl_read_status(ws, stream=None) -> int:

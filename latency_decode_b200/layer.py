@@ -77,6 +77,19 @@ class DecodeLayer:
         dl.check(dl.dl_fc13_swiglu(x2, self.M, self.K, self.wp_13, self.s_13, self.N2, self.ffn_out, self.ws_13,
                                    stream=stream, flags=flags))
 
+    def step_host(self, x_host: torch.Tensor, out_host: torch.Tensor, k_cache, v_cache, seq_lens, stream=None,
+                  flags: int = dl.DL_FLAG_PDL) -> None:
+        """One step whose activations come from, and whose results go to, pinned
+        host memory: x_host is [2, M, K] bf16 bits (x1, x2) from cudaHostAlloc
+        (torch's pin_memory), out_host has the layout of self.out_buf.  The two
+        transfers are kernels of the same PDL chain (dl_copy), so the QKV GEMM
+        streams its weights while the activations arrive."""
+        if not hasattr(self, "x_dev"):
+            self.x_dev = torch.empty((2, self.M, self.K), dtype=torch.int16, device=self.device)
+        dl.check(dl.dl_copy(x_host, self.x_dev, self.x_dev.numel() * 2, stream=stream, flags=flags))
+        self.step(self.x_dev[0], self.x_dev[1], k_cache, v_cache, seq_lens, stream=stream, flags=flags)
+        dl.check(dl.dl_copy(self.out_buf, out_host, self.out_buf.numel() * 2, stream=stream, flags=flags))
+
     def read_status(self, stream=None) -> None:
         for ws in (self.ws_qkv, self.ws_attn, self.ws_13):
             if ws is not None:

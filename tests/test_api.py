@@ -251,3 +251,10 @@ def test_fp8kv_attention_argument_errors():
     assert f(**{**a, "cluster_size": 3}) == dl.DL_ERR_INVALID_ARG
     assert f(**{**a, "ws_bytes": 255}) == dl.DL_ERR_WORKSPACE
     assert dl.dl_decode_attn_fp8kv_workspace_bytes(1, 1, 8, 2, 64, 256, 8) == 0
+
+
+def test_copy_argument_errors():
+    assert dl.dl_copy(None, FAKE, 16, 0, 0) == dl.DL_ERR_INVALID_ARG
+    assert dl.dl_copy(FAKE, FAKE + 4096, 17, 0, 0) == dl.DL_ERR_ALIGNMENT
+    assert dl.dl_copy(FAKE + 8, FAKE + 4096, 16, 0, 0) == dl.DL_ERR_ALIGNMENT
+    assert dl.dl_copy(FAKE, FAKE + 16, 64, 0, 0) == dl.DL_ERR_INVALID_ARG  # overlap
