@@ -45,6 +45,9 @@ def parse_args():
     p.add_argument("--no-full-layer", action="store_true", help="skip the whole-layer (7-kernel) figure")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="only run this many direct-launch layer steps (for a profiler), print no JSON line")
+    p.add_argument("--profile-next", type=int, default=0,
+                   help="only run this many direct-launch whole-layer steps, FP8-cache attention calls and "
+                        "verification calls (for a profiler), print no JSON line")
     return p.parse_args()
 
 
@@ -287,6 +290,120 @@ def make_full_layers(wl, R, seed_base, device, cluster):
     return out
 
 
+def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, capture_fn, graph_steps_fn, peak):
+    """Per-call device time of the rows beyond the headline chain, each timed the
+    way the headline kernels are (graphs of back-to-back calls over more than
+    3x L2 of distinct inputs), with its algorithmic bytes and roofline fraction."""
+    import torch
+    from latency_decode_b200 import dl
+
+    out = {}
+    RF = len(fl)
+
+    def timed_call(fn, reps):
+        for i in range(3):
+            fn(i)
+        gbig = capture_fn(fn, range(reps))
+        graph_steps_fn(2 * reps, gbig, [gbig], reps)
+        n = max(reps, (steps // reps) * reps)
+        return timed_graph_fn(n, gbig, [gbig], reps) * 1e3 / n
+
+    def entry(us, nbytes, extra=None):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        e = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak}
+        e.update(extra or {})
+        return e
+
+    h = lambda: torch.cuda.current_stream().cuda_stream
+    G = RF * max(1, 24 // RF)
+    # NEXT-1: plain projections and the RMSNorm producer
+    def o_proj(i):
+        lay = fl[i % RF][0]
+        dl.check(dl.dl_gemm_e4m3(lay.attn_out, wl.M, wl.k_o, lay.wp["o"], lay.s["o"], wl.K, lay.a, lay.ws_o,
+                                 stream=h()))
+    def fc2(i):
+        lay = fl[i % RF][0]
+        dl.check(dl.dl_gemm_e4m3(lay.f, wl.M, wl.k_fc2, lay.wp["2"], lay.s["2"], wl.K, lay.y, lay.ws_2, stream=h()))
+    def norm(i):
+        lay, kc, vc, x, hres = fl[i % RF]
+        dl.check(dl.dl_add_rmsnorm_quant(x, hres, hres, lay.g1, wl.M, wl.K, 1e-5, lay.ws_qkv, stream=h()))
+    out["o_proj"] = entry(timed_call(o_proj, G), wl.K * wl.k_o)
+    out["fc2"] = entry(timed_call(fc2, G), wl.K * wl.k_fc2)
+    out["add_rmsnorm_quant"] = entry(timed_call(norm, G), 3 * wl.M * wl.K * 2 + wl.M * wl.K,
+                                     {"note": "latency-bound at this size"})
+    # NEXT-3: attention over an e4m3 cache (half the bytes of the bf16 cache)
+    if wl.d == 128:
+        sl_host = seq_lens.cpu().numpy()
+        kv8 = int(sum(2 * wl.Hkv * int(L) * wl.d for L in sl_host))
+        R8 = max(2, -(-3 * 126 * 10**6 // (2 * wl.B * wl.Hkv * wl.Lcap * wl.d)))
+        gen = torch.Generator(device=device).manual_seed(77)
+        caches = [tuple(torch.randint(0, 0x7E, (wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device,
+                                      dtype=torch.uint8) for _ in range(2)) for _ in range(R8)]
+        scales = torch.tensor([0.01, 0.02], dtype=torch.float32, device=device)
+        n = dl.dl_decode_attn_fp8kv_workspace_bytes(wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, wl.Lcap, cluster)
+        wss = [torch.zeros(n, dtype=torch.uint8, device=device) for _ in range(R8)]
+        def attn8(i):
+            r = i % R8
+            lay = fl[i % RF][0]
+            dl.check(dl.dl_decode_attn_fp8kv(lay.qkv, lay.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, caches[r][0],
+                                             caches[r][1], scales, wl.Lcap, seq_lens, 1.0, cluster, lay.attn_out,
+                                             wss[r], stream=h()))
+        out["decode_attn_fp8kv"] = entry(timed_call(attn8, R8 * max(1, 24 // R8)), kv8)
+        for w in wss:
+            dl.check(dl.dl_read_status(w))
+        del caches, wss
+    # NEXT-4: greedy verification over the full vocabulary at this step's B and T
+    from latency_decode_b200 import datagen as dg
+    V = dg.VOCAB
+    per = wl.B * wl.T * V * 2
+    RV = max(2, min(2048, -(-3 * 126 * 10**6 // per)))
+    lg = torch.randn((RV, wl.B, wl.T, V), device=device).to(torch.bfloat16).view(torch.int16)
+    dr = torch.randint(0, V, (wl.B, max(1, wl.T - 1)), device=device, dtype=torch.int32)
+    tid = torch.empty((wl.B, wl.T), dtype=torch.int32, device=device)
+    nacc = torch.empty((wl.B,), dtype=torch.int32, device=device)
+    em = torch.empty((wl.B, wl.T), dtype=torch.int32, device=device)
+    def verify(i):
+        dl.check(dl.dl_spec_verify_greedy(lg[i % RV], wl.B, wl.T, V, dr, tid, nacc, em, None, stream=h()))
+    out["spec_verify_greedy"] = entry(timed_call(verify, RV * max(1, 24 // RV) if RV < 24 else RV), per,
+                                      {"vocab": V})
+    del lg
+    torch.cuda.empty_cache()
+    return out
+
+
+def profile_next_rows(wl, n, seq_lens, device, cluster):
+    """n direct-launch steps of the whole layer, n FP8-cache attention calls and
+    n verification calls over the full vocabulary, on two replicas (the input of
+    an ncu capture of those kernels)."""
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200 import dl
+
+    fl = make_full_layers(wl, 2, 7000, device, cluster)
+    gen = torch.Generator(device=device).manual_seed(78)
+    c8 = [torch.randint(0, 0x7E, (wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device, dtype=torch.uint8)
+          for _ in range(2)]
+    scales = torch.tensor([0.01, 0.02], dtype=torch.float32, device=device)
+    ws8 = torch.zeros(dl.dl_decode_attn_fp8kv_workspace_bytes(wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, wl.Lcap, cluster),
+                      dtype=torch.uint8, device=device)
+    V = dg.VOCAB
+    lg = torch.randn((wl.B, wl.T, V), generator=gen, device=device).to(torch.bfloat16).view(torch.int16)
+    dr = torch.randint(0, V, (wl.B, max(1, wl.T - 1)), generator=gen, device=device, dtype=torch.int32)
+    tid = torch.empty((wl.B, wl.T), dtype=torch.int32, device=device)
+    nacc = torch.empty((wl.B,), dtype=torch.int32, device=device)
+    em = torch.empty((wl.B, wl.T), dtype=torch.int32, device=device)
+    h = torch.cuda.current_stream().cuda_stream
+    for i in range(n):
+        lay, kc, vc, x, hres = fl[i % 2]
+        lay.step(x, hres, kc, vc, seq_lens, stream=h)
+        dl.check(dl.dl_decode_attn_fp8kv(lay.qkv, lay.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, c8[0], c8[1], scales,
+                                         wl.Lcap, seq_lens, 1.0, cluster, lay.attn_out, ws8, stream=h))
+        dl.check(dl.dl_spec_verify_greedy(lg, wl.B, wl.T, V, dr, tid, nacc, em, None, stream=h))
+    for entry in fl:
+        entry[0].read_status(h)
+    dl.check(dl.dl_read_status(ws8, h))
+
+
 def gemm_launches(M, K):
     """Kernels one GEMM entry point launches: the GEMM quantises inputs of up to
     32768 elements itself, larger ones get a quantise kernel first."""
@@ -337,6 +454,11 @@ def run_ours(args):
         layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens,
                        stream=torch.cuda.current_stream().cuda_stream, flags=flags)
 
+    if args.profile_next > 0:  # a short, graph-free run of the rows beyond the headline chain
+        profile_next_rows(wl, args.profile_next, seq_lens, device, cluster)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     if args.profile_steps > 0:  # a short, graph-free run of the chain for a profiler
         for i in range(args.profile_steps):
             step(i)
@@ -472,6 +594,7 @@ def run_ours(args):
 
     # ---- the whole pre-norm layer (adds O_proj, FC2 and both RMSNorm producers) ----
     full = None
+    next_rows = None
     if not args.no_full_layer:
         fbytes = wl.n_qkv * K + wl.K * wl.k_o + wl.N2 * K + wl.K * wl.k_fc2
         RF = max(2, math.ceil(3 * L2_BYTES / (fbytes + 2 * wl.B * wl.Hkv * wl.Lcap * wl.d * 2)))
@@ -504,6 +627,8 @@ def run_ours(args):
                 "launches_per_step": f_launches, "mode": fmode, "replicas": RF,
                 "steps": "add+RMSNorm+quant -> FC_QKV -> attention -> O_proj -> add+RMSNorm+quant -> FC13+SwiGLU "
                          "-> FC2"}
+        next_rows = measure_next_rows(wl, fl, seq_lens, device, cluster, args.steps, timed_graph, capture,
+                                      graph_steps, peak)
         del fl
         torch.cuda.empty_cache()
 
@@ -582,6 +707,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "gpu_launches": (2 * gl + 1) * args.steps,
         "full_layer": full,
+        "next_rows": next_rows,
         "clocks": clk,
         "replicas": R,
     }
