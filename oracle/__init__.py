@@ -301,15 +301,16 @@ def decode_attn(q, q_stride, B, T, Hq, Hkv, d, k_cache, v_cache, seq_lens, scale
     return out
 
 
-def decode_attn_fp8kv(q, q_stride, B, T, Hq, Hkv, d, k_codes, v_codes, seq_lens, scale, s_k, s_v) -> np.ndarray:
-    """As decode_attn, with e4m3 caches (uint8 [B, Hkv, Lcap, d]) and per-tensor scales."""
+def decode_attn_fp8kv(q, q_stride, B, T, Hq, Hkv, d, k_codes, vt_codes, seq_lens, scale, s_k, s_v) -> np.ndarray:
+    """As decode_attn, with e4m3 caches and per-tensor scales: k_codes uint8
+    [B, Hkv, Lcap, d], vt_codes uint8 [B, Hkv, d, Lcap] (V stored transposed)."""
     lib = _load()
     q = _c(q, np.uint16)
     k = _c(k_codes, np.uint8)
-    v = _c(v_codes, np.uint8)
+    v = _c(vt_codes, np.uint8)
     sl = _c(seq_lens, np.int32)
     Lcap = k.shape[2]
-    assert k.shape == (B, Hkv, Lcap, d) and v.shape == k.shape and sl.shape == (B,)
+    assert k.shape == (B, Hkv, Lcap, d) and v.shape == (B, Hkv, d, Lcap) and sl.shape == (B,)
     out = np.zeros((B, T, Hq, d), dtype=np.float64)
     lib.oracle_decode_attn_fp8kv(_ptr(q), int(q_stride), B, T, Hq, Hkv, d, _ptr(k), _ptr(v), Lcap, _ptr(sl),
                                  float(scale), float(s_k), float(s_v), _ptr(out))

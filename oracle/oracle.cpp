@@ -341,7 +341,7 @@ void oracle_decode_attn(const uint16_t* q, long long q_stride, int B, int T, int
 }
 
 void oracle_decode_attn_fp8kv(const uint16_t* q, long long q_stride, int B, int T, int Hq, int Hkv,
-                              int d, const uint8_t* k, const uint8_t* v, int Lcap,
+                              int d, const uint8_t* k, const uint8_t* v_t, int Lcap,
                               const int32_t* seq_lens, float scale, float s_k, float s_v,
                               double* out) {
   const int g = Hq / Hkv;
@@ -367,7 +367,8 @@ void oracle_decode_attn_fp8kv(const uint16_t* q, long long q_stride, int B, int 
         for (int j = 0; j < visible; ++j) {
           const double p = std::exp(s[j] - mx);
           l += p;
-          for (int i = 0; i < d; ++i) o[i] += p * (static_cast<double>(s_v) * kE4m3.v[v[head + static_cast<size_t>(j) * d + i]]);
+          for (int i = 0; i < d; ++i)  // v_t is [d][Lcap] per head: element (key j, dim i) at i*Lcap + j
+            o[i] += p * (static_cast<double>(s_v) * kE4m3.v[v_t[head + static_cast<size_t>(i) * Lcap + j]]);
         }
         double* dst = out + ((static_cast<size_t>(b) * T + t) * Hq + h) * d;
         for (int i = 0; i < d; ++i) dst[i] = l > 0.0 ? o[i] / l : 0.0;

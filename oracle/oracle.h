@@ -143,10 +143,12 @@ void oracle_decode_attn(const uint16_t* q, long long q_stride, int B, int T, int
 /* ---- A3 with an FP8 KV cache ([TC] and [XZY]: FP8 is used for attention as
  * well as for the GEMMs and MoE).  Reading: the cache holds e4m3 codes with one
  * per-tensor scale each for K and V, k = s_k * e4m3(code), v = s_v * e4m3(code);
- * q stays bf16.  Otherwise exactly oracle_decode_attn (same layout, GQA map and
- * bottom-right causal rule); k and v are [B][Hkv][Lcap][d] bytes. */
+ * q stays bf16.  k is [B][Hkv][Lcap][d] bytes as in oracle_decode_attn; the V
+ * cache is stored transposed, v_t [B][Hkv][d][Lcap] (key j, dim i at
+ * i*Lcap + j).  Otherwise exactly oracle_decode_attn (GQA map, bottom-right
+ * causal rule). */
 void oracle_decode_attn_fp8kv(const uint16_t* q, long long q_stride, int B, int T, int Hq, int Hkv,
-                              int d, const uint8_t* k, const uint8_t* v, int Lcap,
+                              int d, const uint8_t* k, const uint8_t* v_t, int Lcap,
                               const int32_t* seq_lens, float scale, float s_k, float s_v,
                               double* out);
 

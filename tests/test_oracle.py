@@ -594,7 +594,8 @@ def test_fp8kv_attention_equals_bf16_attention_on_exactly_representable_caches()
     vc[(vc & 0x7F) == 0x7F] = 0x38
     s_k, s_v = np.float32(2.0 ** -7), np.float32(2.0 ** -5)
     sl = np.int32([96, 37])
-    got = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.125, s_k, s_v)
+    vt = np.ascontiguousarray(vc.transpose(0, 1, 3, 2))  # the FP8 cache stores V as [d][key]
+    got = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vt, sl, 0.125, s_k, s_v)
     kb = dg.bf16_bits((_dequant_torch(kc) * float(s_k)).astype(np.float32))
     vb = dg.bf16_bits((_dequant_torch(vc) * float(s_v)).astype(np.float32))
     assert np.array_equal(_bf16_torch(kb), _dequant_torch(kc) * float(s_k))  # exact in bf16
@@ -611,6 +612,7 @@ def test_fp8kv_scales_enter_as_stated():
     kc = g.integers(0, 0x7E, size=(B, Hkv, Lcap, d)).astype(np.uint8)
     vc = g.integers(0, 0x7E, size=(B, Hkv, Lcap, d)).astype(np.uint8)
     sl = np.int32([50])
-    a = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.5, 0.01, 1.0)
-    b = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vc, sl, 0.25, 0.02, 3.0)
+    vt = np.ascontiguousarray(vc.transpose(0, 1, 3, 2))
+    a = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vt, sl, 0.5, 0.01, 1.0)
+    b = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vt, sl, 0.25, 0.02, 3.0)
     assert np.allclose(b, 3.0 * a, rtol=1e-12)
