@@ -337,8 +337,9 @@ def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, 
         kv8 = int(sum(2 * wl.Hkv * int(L) * wl.d for L in sl_host))
         R8 = max(2, -(-3 * 126 * 10**6 // (2 * wl.B * wl.Hkv * wl.Lcap * wl.d)))
         gen = torch.Generator(device=device).manual_seed(77)
-        caches = [tuple(torch.randint(0, 0x7E, (wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device,
-                                      dtype=torch.uint8) for _ in range(2)) for _ in range(R8)]
+        caches = [tuple(torch.randint(0, 0x7E, shape, generator=gen, device=device, dtype=torch.uint8)
+                        for shape in ((wl.B, wl.Hkv, wl.Lcap, wl.d), (wl.B, wl.Hkv, wl.d, wl.Lcap)))  # K, V^T
+                  for _ in range(R8)]
         scales = torch.tensor([0.01, 0.02], dtype=torch.float32, device=device)
         n = dl.dl_decode_attn_fp8kv_workspace_bytes(wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, wl.Lcap, cluster)
         wss = [torch.zeros(n, dtype=torch.uint8, device=device) for _ in range(R8)]
@@ -381,8 +382,8 @@ def profile_next_rows(wl, n, seq_lens, device, cluster):
 
     fl = make_full_layers(wl, 2, 7000, device, cluster)
     gen = torch.Generator(device=device).manual_seed(78)
-    c8 = [torch.randint(0, 0x7E, (wl.B, wl.Hkv, wl.Lcap, wl.d), generator=gen, device=device, dtype=torch.uint8)
-          for _ in range(2)]
+    c8 = [torch.randint(0, 0x7E, shape, generator=gen, device=device, dtype=torch.uint8)
+          for shape in ((wl.B, wl.Hkv, wl.Lcap, wl.d), (wl.B, wl.Hkv, wl.d, wl.Lcap))]  # K, V^T
     scales = torch.tensor([0.01, 0.02], dtype=torch.float32, device=device)
     ws8 = torch.zeros(dl.dl_decode_attn_fp8kv_workspace_bytes(wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, wl.Lcap, cluster),
                       dtype=torch.uint8, device=device)

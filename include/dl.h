@@ -249,6 +249,28 @@ dl_status dl_add_rmsnorm_quant(const uint16_t* x, const uint16_t* residual, uint
                                size_t ws_bytes, void* stream, unsigned flags);
 
 /* ---------------------------------------------------------------------------
+ * Residual add + RMSNorm + Quantize, then the GEMM that consumes it, in one call.
+ * [XZY] "运算融合" / [NV] fusion list: the (AllReduce +) RMSNorm + Quantize
+ * producer of a GEMM input.  Exactly dl_add_rmsnorm_quant(x, residual, h_out,
+ * gamma, M, K, eps, ws) followed by dl_fc_qkv_scale / dl_fc13_swiglu with
+ * DL_FLAG_XQ_READY and the same ws: two kernels chained under DL_FLAG_PDL, so
+ * the GEMM streams its weights while the producer runs.  (Computing the
+ * producer inside every GEMM CTA instead was measured slower: each CTA re-reads
+ * x, residual and gamma.)  h_out may be x or residual itself but must not
+ * partially overlap either.  The remaining arguments are those of
+ * dl_fc_qkv_scale / dl_fc13_swiglu; x is required.
+ * ------------------------------------------------------------------------- */
+dl_status dl_rmsnorm_fc_qkv_scale(const uint16_t* x, const uint16_t* residual, uint16_t* h_out,
+                                  const uint16_t* gamma, float eps, int M, int K,
+                                  const uint8_t* w_packed, const float* w_scale, int Hq, int Hkv,
+                                  int d, float q_scale, uint16_t* qkv, void* ws, size_t ws_bytes,
+                                  void* stream, unsigned flags);
+dl_status dl_rmsnorm_fc13_swiglu(const uint16_t* x, const uint16_t* residual, uint16_t* h_out,
+                                 const uint16_t* gamma, float eps, int M, int K,
+                                 const uint8_t* w_packed, const float* w_scale, int N2, uint16_t* out,
+                                 void* ws, size_t ws_bytes, void* stream, unsigned flags);
+
+/* ---------------------------------------------------------------------------
  * Split-KV grouped-query decode attention with a cluster DSMEM merge.
  * [XZY] "CUDA 内核优化与融合", item "Attention内核并行优化"; [NV] "CUDA kernel
  * optimisation and fusion": the work is split along the sequence dimension of
@@ -288,19 +310,21 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
  * Split-KV decode attention over an FP8 (e4m3) KV cache.  [TC] and [XZY]
  * (section "CUDA 内核优化与融合" and the FP8 rationale): FP8 is used for
  * attention as well as for the GEMMs and MoE; it halves the KV bytes streamed.
- * Same computation, layout, split, merge and rules as dl_decode_attn, except:
- *   k_cache, v_cache  e4m3 bytes [B][Hkv][Lcap][d] (OCP E4M3 "e4m3fn"), the
- *             cache holding k / s_k and v / s_v
+ * Same computation, split, merge and rules as dl_decode_attn, except:
+ *   k_cache   e4m3 bytes [B][Hkv][Lcap][d] (OCP E4M3 "e4m3fn"), holding k / s_k
+ *   vt_cache  e4m3 bytes [B][Hkv][d][Lcap]: V stored transposed, holding v / s_v
+ *             (key j, dim i of a head at i*Lcap + j)
  *   kv_scale  device float[2] = {s_k, s_v}, the per-tensor cache scales (a
  *             static input: read before the PDL wait)
- * o = softmax(softmax_scale * q (s_k K)^T) (s_v V).  The tile is converted to
- * f16 on chip and the products run in f16 with fp32 accumulation (q and the
- * probabilities are rounded to f16).  Supported: d = 128, (Hq/Hkv)*T <= 32.
- * The workspace rules are those of dl_decode_attn, sized by
- * dl_decode_attn_fp8kv_workspace_bytes.
+ *   Lcap      a multiple of 16 (DL_ERR_ALIGNMENT otherwise)
+ * o = softmax(softmax_scale * q (s_k K)^T) (s_v V).  The MMA operands are
+ * converted to f16 in registers (exact for e4m3) and the products run in f16
+ * with fp32 accumulation (q and the probabilities are rounded to f16).
+ * Supported: d = 128, (Hq/Hkv)*T <= 32.  The workspace rules are those of
+ * dl_decode_attn, sized by dl_decode_attn_fp8kv_workspace_bytes.
  * ------------------------------------------------------------------------- */
 dl_status dl_decode_attn_fp8kv(const uint16_t* q, long long q_token_stride, int B, int T, int Hq,
-                               int Hkv, int d, const uint8_t* k_cache, const uint8_t* v_cache,
+                               int Hkv, int d, const uint8_t* k_cache, const uint8_t* vt_cache,
                                const float* kv_scale, int Lcap, const int32_t* seq_lens,
                                float softmax_scale, int cluster_size, uint16_t* out, void* ws,
                                size_t ws_bytes, void* stream, unsigned flags);

@@ -68,15 +68,37 @@ struct AttnArgs {
   int debug;
 };
 
+// Two e4m3 codes (low byte first) -> f16x2 (low half first); exact, since every
+// e4m3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// 4 bytes at (row, col) of a V^T tile of KT-byte rows as TMA lays it out: the
+// 128-byte swizzle for 128-byte rows, the 64-byte swizzle for 64-byte rows
+// (16-byte chunk index XOR row bits; col is a multiple of 4).
+template <int KT>
+__device__ __forceinline__ uint32_t vt_word(const uint8_t* vt, int row, int col) {
+  static_assert(KT == 64 || KT == 128, "V^T rows of 64 or 128 bytes");
+  const int ch = KT == 128 ? (((col >> 4) ^ row) & 7) : (((col >> 4) ^ (row >> 1)) & 3);
+  return *reinterpret_cast<const uint32_t*>(vt + row * KT + (ch << 4) + (col & 15));
+}
+
 __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
 // F8: the KV cache holds e4m3 codes (one byte per element) with per-tensor
-// scales s_k, s_v.  The ring then carries half the bytes; each consumer warp
-// converts its 16 keys of a tile to f16 in a private staging buffer laid out
-// like a bf16 tile (so the ldmatrix paths are shared), frees the ring slot at
-// once, and runs the MMAs in f16 (Q and P are converted to f16 as well).
+// scales s_k, s_v; K is [key][d] and V is stored transposed, [d][key].  The
+// ring carries half the bytes, and the MMA operands are converted to f16 in
+// registers straight from the TMA-landed tiles (cvt e4m3x2 -> f16x2), with no
+// staging pass: inside each warp's 16 keys the MMA key index r stands for the
+// physical key pi(r) = 4*((r%8)/2) + 2*(r/8) + r%2, and inside each k-step the
+// d index of thread t for element e stands for physical d = 32t + 4ks + e.
+// Both are fixed permutations of a dot product's terms (Q's fragments use the
+// same d map; the causal mask uses pi), chosen so that every fragment a thread
+// needs is 4 (V^T) or 16 (K) contiguous bytes.  Q and P are rounded to f16.
 template <int D, int NT, int W, bool F8>
 __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -89,15 +111,12 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   constexpr int HALF_BYTES = kAttnKT * 128;   // kAttnKT keys x 128 bytes
   constexpr int KV_BYTES = F8 ? kAttnKT * D : HALVES * HALF_BYTES;  // one of K, V in a stage
   constexpr int STAGE_BYTES = 2 * KV_BYTES;
-  constexpr int STG_HALF = 16 * 128;          // f16 staging: 16 keys x 64 d per half
-  constexpr int STG_BYTES = F8 ? 2 * HALVES * STG_HALF : 0;  // per consumer warp: K halves, V halves
   constexpr int KS = D / 16;                  // MMA k-steps over d, and m-tiles of d
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
-  uint8_t* stg_all = ring + a.stages * STAGE_BYTES;                           // [W][STG_BYTES]
-  uint2* qs = reinterpret_cast<uint2*>(stg_all + kAttnConsumers * STG_BYTES);  // [KS][NT][32]
+  uint2* qs = reinterpret_cast<uint2*>(ring + a.stages * STAGE_BYTES);        // [KS][NT][32]
   uint8_t* recv_base = smem + a.recv_off;                                      // DSMEM receive buffer
   uint64_t* bars = reinterpret_cast<uint64_t*>(qs + KS * NT * 32);
   int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages);
@@ -200,9 +219,9 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         const uint32_t fb = full0 + 8u * s;
         mbar_arrive_expect_tx(fb, STAGE_BYTES);
         const int key0 = lo + i * kAttnKT;
-        if (F8) {  // one 128-byte e4m3 row per key: a single box per tensor
+        if (F8) {  // K: KT rows of 128 bytes; V^T: 128 rows (d) of KT bytes
           tma_load_3d(st, &tk, 0, key0, z, fb);
-          tma_load_3d(st + KV_BYTES, &tv, 0, key0, z, fb);
+          tma_load_3d(st + KV_BYTES, &tv, key0, 0, z, fb);
         } else {
 #pragma unroll
           for (int h = 0; h < HALVES; ++h) {
@@ -237,11 +256,14 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         const int hq = hk * a.G + rho % a.G;
         const uint16_t* qrow =
             a.q + (static_cast<long long>(b) * a.T + t) * a.q_stride + static_cast<long long>(hq) * D;
-        v.x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
-        v.y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
-        if (F8) {  // bf16 pairs -> f16 pairs (the f16 MMA needs both operands in f16)
-          v.x = pack_f16x2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u));
-          v.y = pack_f16x2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+        if (F8) {  // k-step ks, thread t: physical d = 32t + 4ks + e; bf16 -> f16
+          const int d0 = 32 * (ln & 3) + 4 * ks;
+          const uint32_t w0 = ld_b32(qrow + d0), w1 = ld_b32(qrow + d0 + 2);
+          v.x = pack_f16x2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
+          v.y = pack_f16x2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
+        } else {
+          v.x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
+          v.y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
         }
       }
       qs[f] = v;
@@ -250,7 +272,9 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
 
     // F8: the cache holds k / s_k, so the logits take s_k into their scale
     const float scale_log2 = F8 ? a.scale_log2 * __ldg(a.kv_scale) : a.scale_log2;
-    uint8_t* stg = stg_all + warp * STG_BYTES;
+    // F8: physical key offsets (within the warp's 16) of MMA rows g and g+8
+    const int pA = F8 ? 4 * (g >> 1) + (g & 1) : g;
+    const int pB = F8 ? pA + 2 : g + 8;
 
     int lim[NT][2];  // last visible key of the rows this thread accumulates
 #pragma unroll
@@ -271,72 +295,58 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
       ok = __all_sync(0xffffffffu, ok);  // the warp-wide MMA path below needs a uniform decision
       const int key_base = lo + i * kAttnKT + warp * 16;
-      bool released = false;
-      if (F8 && ok && key_base < hi) {
-        // e4m3 rows of this warp's 16 keys -> f16 staging in the swizzled bf16-tile
-        // layout; lane = (key r, 64-d half hf), 4 chunks of 16 codes each for K and V.
-        const int r = lane >> 1;
-        const int hf = lane & 1;
-        const int rr = warp * 16 + r;  // row within the stage
-        const uint8_t* kst = ring + s * STAGE_BYTES;
-#pragma unroll
-        for (int t2 = 0; t2 < 2; ++t2) {  // K, then V
-          const uint8_t* src = kst + t2 * KV_BYTES + rr * 128;
-          uint8_t* dst = stg + t2 * HALVES * STG_HALF + hf * STG_HALF + r * 128;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = hf * 4 + c4;  // 16-byte chunk of the 128-byte row: d = 16c .. 16c+15
-            const uint4 u = *reinterpret_cast<const uint4*>(src + ((c ^ (rr & 7)) << 4));
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            uint32_t hv[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __half2_raw lo2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[e] & 0xFFFFu), __NV_E4M3);
-              const __half2_raw hi2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[e] >> 16), __NV_E4M3);
-              hv[2 * e] = static_cast<uint32_t>(lo2.x) | (static_cast<uint32_t>(lo2.y) << 16);
-              hv[2 * e + 1] = static_cast<uint32_t>(hi2.x) | (static_cast<uint32_t>(hi2.y) << 16);
-            }
-            *reinterpret_cast<uint4*>(dst + (((2 * c4) ^ (r & 7)) << 4)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4*>(dst + (((2 * c4 + 1) ^ (r & 7)) << 4)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8u * s);  // the ring slot is free: staging holds the tile
-        released = true;
-      }
       if (ok && key_base < hi) {
-        // F8: this warp's staging holds rows 0..15; bf16: the ring holds rows warp*16 ..
-        const int row0 = F8 ? 0 : warp * 16;
-        const int half_bytes = F8 ? STG_HALF : HALF_BYTES;
-        const uint32_t kbase = F8 ? smem_u32(stg) : smem_u32(ring + s * STAGE_BYTES);
-        const uint32_t vbase = kbase + HALVES * half_bytes;
+        const uint32_t kbase = smem_u32(ring + s * STAGE_BYTES);
+        const uint32_t vbase = kbase + KV_BYTES;
         // ---- S^T[16 keys x 8*NT rows] = K . Q^T ----
         float sc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int c = 0; c < 4; ++c) sc[nt][c] = 0.0f;
-        {
+        if (F8) {
+          // rows pi(g), pi(g+8) of K: bytes 32t .. 32t+31 (chunks 2t, 2t+1) hold
+          // e = 0..3 of k-steps 0..7 for this thread
+          const int rA = warp * 16 + pA, rB = warp * 16 + pB;
+          const uint8_t* kt = ring + s * STAGE_BYTES;
+          uint4 kA[2], kB[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            kA[h] = *reinterpret_cast<const uint4*>(kt + rA * 128 + (((2 * q4 + h) ^ (rA & 7)) << 4));
+            kB[h] = *reinterpret_cast<const uint4*>(kt + rB * 128 + (((2 * q4 + h) ^ (rB & 7)) << 4));
+          }
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint32_t wA = (&kA[ks >> 2].x)[ks & 3];
+            const uint32_t wB = (&kB[ks >> 2].x)[ks & 3];
+            const uint32_t a0 = e4m3x2_to_f16x2(wA & 0xFFFFu), a2 = e4m3x2_to_f16x2(wA >> 16);
+            const uint32_t a1 = e4m3x2_to_f16x2(wB & 0xFFFFu), a3 = e4m3x2_to_f16x2(wB >> 16);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint2 qf = qs[(ks * NT + nt) * 32 + lane];
+              mma_f16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
+            }
+          }
+        } else {
           const int j = lane >> 3;
-          const int key_l = row0 + (j & 1) * 8 + (lane & 7);
+          const int key_l = warp * 16 + (j & 1) * 8 + (lane & 7);
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             const int half = ks >> 2;
             const int ch = (ks & 3) * 2 + (j >> 1);
-            const uint32_t addr = kbase + half * half_bytes + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
+            const uint32_t addr = kbase + half * HALF_BYTES + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const uint2 qf = qs[(ks * NT + nt) * 32 + lane];
-              if (F8) mma_f16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
-              else mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
+              mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf.x, qf.y);
             }
           }
         }
         // ---- online softmax (log2 domain) ----
-        const int kA = key_base + g;
-        const int kB = kA + 8;
+        const int kA = key_base + pA;  // physical keys of MMA rows g and g+8
+        const int kB = key_base + pB;
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -373,26 +383,38 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           pb[nt][1] = movmatrix_t(F8 ? pack_f16x2(p[2], p[3]) : pack_bf16x2(p[2], p[3]));
         }
         // ---- O^T[d x rows] += V^T . P^T ----
-        {
+        if (F8) {
+          // V^T rows 16mt+g and 16mt+g+8 (d), bytes warp*16 + 4t .. +3 = MMA keys
+          // 2t, 2t+1 (e = 0, 1) and 2t+8, 2t+9 (e = 2, 3)
+          const uint8_t* vt = ring + s * STAGE_BYTES + KV_BYTES;
+          const int col = warp * 16 + 4 * q4;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            const int r0 = 16 * mt + g, r1 = r0 + 8;
+            const uint32_t w0 = vt_word<kAttnKT>(vt, r0, col);
+            const uint32_t w1 = vt_word<kAttnKT>(vt, r1, col);
+            const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xFFFFu), a2 = e4m3x2_to_f16x2(w0 >> 16);
+            const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xFFFFu), a3 = e4m3x2_to_f16x2(w1 >> 16);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          }
+        } else {
           const int j = lane >> 3;
-          const int key_l = row0 + (j >> 1) * 8 + (lane & 7);
+          const int key_l = warp * 16 + (j >> 1) * 8 + (lane & 7);
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
             const int half = mt >> 2;
             const int ch = (mt & 3) * 2 + (j & 1);
-            const uint32_t addr = vbase + half * half_bytes + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
+            const uint32_t addr = vbase + half * HALF_BYTES + key_l * 128 + ((ch ^ (key_l & 7)) << 4);
             uint32_t a0, a1, a2, a3;
             ldsm_x4_t(addr, a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              if (F8) mma_f16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-              else mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-            }
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
           }
         }
       }
-      __syncwarp();  // (F8) every lane is done reading the staging before it is refilled
-      if (!released && lane == 0) mbar_arrive(empty0 + 8u * s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8u * s);
     }
     // full row sums: add the partial sums of the 8 lanes that share a row
 #pragma unroll
@@ -590,17 +612,27 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// K or V cache [BH][Lcap][d] as a 3-D tensor map with 128-byte rows per box:
-// bf16 elements in boxes of 64 (two boxes per key for d = 128), or e4m3 bytes
-// in one box of d = 128.
-static bool encode_kv_map(CUtensorMap* m, const void* base, int d, int Lcap, int BH, int kt, bool fp8) {
+// A cache as a 3-D tensor map.  [BH][Lcap][d] with 128-byte rows per box: bf16
+// in boxes of 64 elements (two per key for d = 128), or e4m3 in one box of
+// d = 128 bytes.  transposed (the e4m3 V^T cache, [BH][d][Lcap]): boxes of d
+// rows of kt bytes (128: 128-byte swizzle; 64: 64-byte swizzle).
+static bool encode_kv_map(CUtensorMap* m, const void* base, int d, int Lcap, int BH, int kt, bool fp8,
+                          bool transposed) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t esz = fp8 ? 1 : 2;
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (transposed) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(Lcap), static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(Lcap), static_cast<cuuint64_t>(Lcap) * d};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kt), static_cast<cuuint32_t>(d), 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, kt == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Lcap), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz, static_cast<cuuint64_t>(Lcap) * d * esz};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(kt), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -627,14 +659,13 @@ struct AttnPlan {
 template <int D, int NT, int W, bool F8>
 static AttnPlan attn_plan(int R, int S) {
   constexpr int STAGE_BYTES = F8 ? 2 * (16 * W) * D : 2 * (D / 64) * (16 * W) * 128;
-  constexpr int STG = F8 ? W * 2 * (D / 64) * 16 * 128 : 0;  // f16 staging of all consumer warps
   const int merge_bytes = (W * R * D + 2 * W * R) * 4;
   const int I = R * (D / 4);
   const int Q = (I + S - 1) / S;
   const int recv_bytes = S * Q * (16 + 8);
   const int qs_bytes = (D / 16) * NT * 32 * 8;
   auto smem_for = [&](int st) {
-    return 1024 + st * STAGE_BYTES + STG + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16;
+    return 1024 + st * STAGE_BYTES + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16;
   };
   int stages = D == 128 ? 3 : 6;
   // W = 4 is chosen to put two CTAs on each SM: give up ring depth (down to
@@ -644,11 +675,11 @@ static AttnPlan attn_plan(int R, int S) {
     stages = 6;
     while (stages > 2 && smem_for(stages) > 232448) --stages;
   }
-  while (stages * STAGE_BYTES + STG < merge_bytes) ++stages;  // the merge reuses ring + staging
+  while (stages * STAGE_BYTES < merge_bytes) ++stages;  // the merge reuses the drained ring
   AttnPlan pl;
   pl.stages = stages;
   pl.smem = smem_for(stages);
-  pl.recv_off = ((stages * STAGE_BYTES + STG + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
+  pl.recv_off = ((stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
   return pl;
 }
 
@@ -785,8 +816,8 @@ cudaError_t launch_attn(const AttnLaunch& p, cudaStream_t s) {
   const int W = attn_warps(p.cluster, static_cast<long long>(p.B) * p.Hkv * p.cluster);
   const int kt = 16 * W;  // keys per stage of the chosen variant
   CUtensorMap tk, tv;
-  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8) ||
-      !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8))
+  if (!encode_kv_map(&tk, p.k, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8, false) ||
+      !encode_kv_map(&tv, p.v, p.d, p.Lcap, p.B * p.Hkv, kt, p.fp8, p.fp8))
     return cudaErrorInvalidValue;
   AttnArgs a;
   a.q = p.q;

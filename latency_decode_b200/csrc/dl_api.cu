@@ -135,11 +135,26 @@ dl_status dl_pack_fp8_weight(const uint8_t* w_nk, uint8_t* w_packed, int N, int 
   return cuda_status(dl::launch_pack(w_nk, w_packed, N, K, kind, static_cast<cudaStream_t>(stream)));
 }
 
+struct NormSpec {  // residual add + RMSNorm ahead of the GEMM (gamma == null: none)
+  const uint16_t* residual = nullptr;
+  uint16_t* h_out = nullptr;
+  const uint16_t* gamma = nullptr;
+  float eps = 0.0f;
+};
+
 static dl_status run_dense_gemm(const uint16_t* x, int M, int K, const uint8_t* w_packed, const float* w_scale,
                                 int N, bool swiglu, int q_cols, float q_scale, uint16_t* out, void* ws,
-                                void* stream, unsigned flags) {
+                                void* stream, unsigned flags, const NormSpec& norm = NormSpec()) {
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool pdl = (flags & DL_FLAG_PDL) != 0;
+  if (norm.gamma != nullptr) {
+    // The producer of the input as its own kernel, PDL-chained ahead of the GEMM
+    // (computing it inside every GEMM CTA measured slower: each re-reads x, r and gamma).
+    cudaError_t e = dl::launch_add_rmsnorm_quant(x, norm.residual, norm.h_out, norm.gamma, M, K, norm.eps,
+                                                 dl::ws_xq(ws), dl::ws_sx(ws), s, pdl);
+    if (e != cudaSuccess) return cuda_status(e);
+    flags |= DL_FLAG_XQ_READY;
+  }
   // Small inputs are quantised inside the GEMM (one launch); larger ones by the
   // cluster quantise kernel first.  Both write x_q and s_x to the workspace.
   // With DL_FLAG_XQ_READY a producer kernel (dl_add_rmsnorm_quant) has
@@ -268,6 +283,70 @@ dl_status dl_gemm_e4m3(const uint16_t* x, int M, int K, const uint8_t* w_packed,
   return run_dense_gemm(x, M, K, w_packed, w_scale, N, false, 0, 1.0f, out, ws, stream, flags);
 }
 
+static dl_status check_norm_spec(const uint16_t* x, const uint16_t* residual, const uint16_t* h_out,
+                                 const uint16_t* gamma, int M, int K, float eps) {
+  if (x == nullptr || gamma == nullptr) return DL_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || !(eps < 3.0e38f)) return DL_ERR_INVALID_ARG;
+  if (M > 64 || static_cast<long long>(M) * K > 64ll * 8192) return DL_ERR_UNSUPPORTED;
+  if (!aligned(residual, 16) || !aligned(h_out, 16) || !aligned(gamma, 16)) return DL_ERR_ALIGNMENT;
+  // h_out may be x or residual itself (in-place update), but no partial overlap
+  const uintptr_t bytes = static_cast<uintptr_t>(M) * static_cast<uintptr_t>(K) * 2u;
+  if (h_out != nullptr) {
+    const uintptr_t hb = reinterpret_cast<uintptr_t>(h_out);
+    for (const void* p : {static_cast<const void*>(x), static_cast<const void*>(residual)}) {
+      const uintptr_t pb = reinterpret_cast<uintptr_t>(p);
+      if (p != nullptr && pb != hb && pb < hb + bytes && hb < pb + bytes) return DL_ERR_INVALID_ARG;
+    }
+  }
+  return DL_OK;
+}
+
+dl_status dl_rmsnorm_fc_qkv_scale(const uint16_t* x, const uint16_t* residual, uint16_t* h_out,
+                                  const uint16_t* gamma, float eps, int M, int K, const uint8_t* w_packed,
+                                  const float* w_scale, int Hq, int Hkv, int d, float q_scale, uint16_t* qkv,
+                                  void* ws, size_t ws_bytes, void* stream, unsigned flags) {
+  flags &= ~DL_FLAG_XQ_READY;
+  dl_status st = check_gemm_common(x, M, K, w_packed, w_scale, qkv, flags);
+  if (st != DL_OK) return st;
+  st = check_norm_spec(x, residual, h_out, gamma, M, K, eps);
+  if (st != DL_OK) return st;
+  if (Hq < 1 || Hkv < 0 || d < 1) return DL_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(Hq + 2 * Hkv) * d;
+  if (N % 128 != 0 || N > (1ll << 24)) return DL_ERR_UNSUPPORTED;
+  if (forced_split(flags) > 8) return DL_ERR_INVALID_ARG;
+  st = check_ws(ws, ws_bytes, dl_workspace_bytes(M, K));
+  if (st != DL_OK) return st;
+  NormSpec ns;
+  ns.residual = residual;
+  ns.h_out = h_out;
+  ns.gamma = gamma;
+  ns.eps = eps;
+  return run_dense_gemm(x, M, K, w_packed, w_scale, static_cast<int>(N), false, Hq * d, q_scale, qkv, ws, stream,
+                        flags, ns);
+}
+
+dl_status dl_rmsnorm_fc13_swiglu(const uint16_t* x, const uint16_t* residual, uint16_t* h_out,
+                                 const uint16_t* gamma, float eps, int M, int K, const uint8_t* w_packed,
+                                 const float* w_scale, int N2, uint16_t* out, void* ws, size_t ws_bytes,
+                                 void* stream, unsigned flags) {
+  flags &= ~DL_FLAG_XQ_READY;
+  dl_status st = check_gemm_common(x, M, K, w_packed, w_scale, out, flags);
+  if (st != DL_OK) return st;
+  st = check_norm_spec(x, residual, h_out, gamma, M, K, eps);
+  if (st != DL_OK) return st;
+  if (N2 < 256) return DL_ERR_INVALID_ARG;
+  if (N2 % 256 != 0) return DL_ERR_UNSUPPORTED;
+  if (forced_split(flags) > 8) return DL_ERR_INVALID_ARG;
+  st = check_ws(ws, ws_bytes, dl_workspace_bytes(M, K));
+  if (st != DL_OK) return st;
+  NormSpec ns;
+  ns.residual = residual;
+  ns.h_out = h_out;
+  ns.gamma = gamma;
+  ns.eps = eps;
+  return run_dense_gemm(x, M, K, w_packed, w_scale, N2, true, 0, 1.0f, out, ws, stream, flags, ns);
+}
+
 dl_status dl_add_rmsnorm_quant(const uint16_t* x, const uint16_t* residual, uint16_t* h_out, const uint16_t* gamma,
                                int M, int K, float eps, void* ws, size_t ws_bytes, void* stream, unsigned flags) {
   if (x == nullptr || gamma == nullptr) return DL_ERR_INVALID_ARG;
@@ -325,6 +404,7 @@ static dl_status run_attn(const uint16_t* q, long long q_token_stride, int B, in
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
       !aligned(seq_lens, 4) || !aligned(kv_scale, 4))
     return DL_ERR_ALIGNMENT;
+  if (fp8 && Lcap % 16 != 0) return DL_ERR_ALIGNMENT;  // the V^T rows (Lcap bytes) are a TMA stride
   dl_status st = check_ws(ws, ws_bytes, dl_workspace_bytes(0, 0));
   if (st != DL_OK) return st;
   dl::AttnLaunch a{};
@@ -361,10 +441,10 @@ dl_status dl_decode_attn(const uint16_t* q, long long q_token_stride, int B, int
 }
 
 dl_status dl_decode_attn_fp8kv(const uint16_t* q, long long q_token_stride, int B, int T, int Hq, int Hkv, int d,
-                               const uint8_t* k_cache, const uint8_t* v_cache, const float* kv_scale, int Lcap,
+                               const uint8_t* k_cache, const uint8_t* vt_cache, const float* kv_scale, int Lcap,
                                const int32_t* seq_lens, float softmax_scale, int cluster_size, uint16_t* out,
                                void* ws, size_t ws_bytes, void* stream, unsigned flags) {
-  return run_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, true, kv_scale, Lcap, seq_lens,
+  return run_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, vt_cache, true, kv_scale, Lcap, seq_lens,
                   softmax_scale, cluster_size, out, ws, ws_bytes, stream, flags);
 }
 

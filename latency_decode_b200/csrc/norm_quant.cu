@@ -40,58 +40,6 @@ struct NormQuantArgs {
   float eps;
 };
 
-__device__ __forceinline__ float nq_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float nq_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// bf16 round-to-nearest-even of the fp32 sum of two bf16 pairs, packed.  The
-// fp32 sum of two bf16 values is exact unless their exponents differ by more
-// than 16, and then the smaller operand is below half an ulp of the result's
-// bf16 grid, so one further rounding to bf16 equals rounding the exact sum.
-__device__ __forceinline__ uint32_t add2_bf16(uint32_t a, uint32_t b) {
-  const __nv_bfloat162 s = __floats2bfloat162_rn(__fadd_rn(nq_lo(a), nq_lo(b)), __fadd_rn(nq_hi(a), nq_hi(b)));
-  return *reinterpret_cast<const uint32_t*>(&s);
-}
-
-__device__ __forceinline__ uint4 add8_bf16(uint4 a, uint4 b) {
-  return make_uint4(add2_bf16(a.x, b.x), add2_bf16(a.y, b.y), add2_bf16(a.z, b.z), add2_bf16(a.w, b.w));
-}
-
-__device__ __forceinline__ float sumsq8(uint4 u) {
-  float s = 0.0f;
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    s = __fmaf_rn(nq_lo(w[i]), nq_lo(w[i]), s);
-    s = __fmaf_rn(nq_hi(w[i]), nq_hi(w[i]), s);
-  }
-  return s;
-}
-
-// y = (h * rs) * gamma for 8 values; returns max |y| and fills y.
-__device__ __forceinline__ float norm8(uint4 h, uint4 g, float rs, float* y) {
-  const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
-  const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    y[2 * i] = __fmul_rn(__fmul_rn(nq_lo(hw[i]), rs), nq_lo(gw[i]));
-    y[2 * i + 1] = __fmul_rn(__fmul_rn(nq_hi(hw[i]), rs), nq_hi(gw[i]));
-    m = fmaxf(m, fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1])));
-  }
-  return m;
-}
-
-__device__ __forceinline__ uint2 quant8(const float* y, float inv) {
-  uint32_t q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(
-        make_float2(__fmul_rn(y[2 * i], inv), __fmul_rn(y[2 * i + 1], inv)), __NV_SATFINITE, __NV_E4M3);
-    q[i] = static_cast<uint32_t>(p);
-  }
-  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
-}
-
 // h of vector v again, beyond the register set: from h_out when this thread
 // stored it there (whatever h_out aliases), else recomputed from x and r.
 __device__ __forceinline__ uint4 reload_h(const uint4* xv, const uint4* rv, const uint4* hv, int v) {

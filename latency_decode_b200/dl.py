@@ -51,6 +51,8 @@ _SIGNATURES = {
     "dl_gemm_e4m3": (_I, [_P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
     "dl_moe_gemm_grouped": (_I, [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
     "dl_add_rmsnorm_quant": (_I, [_P, _P, _P, _P, _I, _I, _F, _P, _SZ, _P, _U]),
+    "dl_rmsnorm_fc_qkv_scale": (_I, [_P, _P, _P, _P, _F, _I, _I, _P, _P, _I, _I, _I, _F, _P, _P, _SZ, _P, _U]),
+    "dl_rmsnorm_fc13_swiglu": (_I, [_P, _P, _P, _P, _F, _I, _I, _P, _P, _I, _P, _P, _SZ, _P, _U]),
     "dl_spec_verify_greedy": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _U]),
     "dl_decode_attn": (_I, [_P, _LL, _I, _I, _I, _I, _I, _P, _P, _I, _P, _F, _I, _P, _P, _SZ, _P, _U]),
     "dl_decode_attn_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
@@ -169,6 +171,20 @@ def dl_spec_verify_greedy(logits, B, T, V, draft_ids, target_ids, n_accepted, em
                                        _ptr(emitted), _ptr(seq_lens), _stream(stream), flags)
 
 
+def dl_rmsnorm_fc_qkv_scale(x, residual, h_out, gamma, eps, M, K, w_packed, w_scale, Hq, Hkv, d, q_scale, qkv, ws,
+                            ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
+    return lib().dl_rmsnorm_fc_qkv_scale(_ptr(x), _ptr(residual), _ptr(h_out), _ptr(gamma), float(eps), M, K,
+                                         _ptr(w_packed), _ptr(w_scale), Hq, Hkv, d, float(q_scale), _ptr(qkv),
+                                         _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
+def dl_rmsnorm_fc13_swiglu(x, residual, h_out, gamma, eps, M, K, w_packed, w_scale, N2, out, ws, ws_bytes=None,
+                           stream=None, flags=DL_FLAG_PDL) -> int:
+    return lib().dl_rmsnorm_fc13_swiglu(_ptr(x), _ptr(residual), _ptr(h_out), _ptr(gamma), float(eps), M, K,
+                                        _ptr(w_packed), _ptr(w_scale), N2, _ptr(out), _ptr(ws),
+                                        _nbytes(ws, ws_bytes), _stream(stream), flags)
+
+
 def dl_decode_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, Lcap, seq_lens, softmax_scale,
                    cluster_size, out, ws, ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
     return lib().dl_decode_attn(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(v_cache),
@@ -176,9 +192,9 @@ def dl_decode_attn(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, Lcap, 
                                 _nbytes(ws, ws_bytes), _stream(stream), flags)
 
 
-def dl_decode_attn_fp8kv(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, v_cache, kv_scale, Lcap, seq_lens,
+def dl_decode_attn_fp8kv(q, q_token_stride, B, T, Hq, Hkv, d, k_cache, vt_cache, kv_scale, Lcap, seq_lens,
                          softmax_scale, cluster_size, out, ws, ws_bytes=None, stream=None, flags=DL_FLAG_PDL) -> int:
-    return lib().dl_decode_attn_fp8kv(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(v_cache),
+    return lib().dl_decode_attn_fp8kv(_ptr(q), int(q_token_stride), B, T, Hq, Hkv, d, _ptr(k_cache), _ptr(vt_cache),
                                       _ptr(kv_scale), Lcap, _ptr(seq_lens), float(softmax_scale), cluster_size,
                                       _ptr(out), _ptr(ws), _nbytes(ws, ws_bytes), _stream(stream), flags)
 

@@ -99,18 +99,17 @@ class DecodeLayer:
 class FullDecodeLayer:
     """The whole pre-norm decode layer of a dense model on one GPU:
 
-        h  <- x + h;  x1 = RMSNorm(h) * g1 -> e4m3          (dl_add_rmsnorm_quant)
-        qkv = FC_QKV(x1) with the Q columns scaled          (dl_fc_qkv_scale, x_q from the norm)
-        o   = attention(q, K cache, V cache)                (dl_decode_attn, q read in place)
-        a   = O_proj(o)                                     (dl_gemm_e4m3)
-        h  <- a + h;  x2 = RMSNorm(h) * g2 -> e4m3          (dl_add_rmsnorm_quant)
-        f   = SwiGLU(FC13(x2))                              (dl_fc13_swiglu, x_q from the norm)
-        y   = FC2(f)                                        (dl_gemm_e4m3)
+        h1 = x + h;  qkv = FC_QKV(RMSNorm(h1) * g1)         (dl_rmsnorm_fc_qkv_scale)
+        o  = attention(q, K cache, V cache)                 (dl_decode_attn, q read in place)
+        a  = O_proj(o)                                      (dl_gemm_e4m3)
+        h  <- a + h1;  f = SwiGLU(FC13(RMSNorm(h) * g2))    (dl_rmsnorm_fc13_swiglu)
+        y  = FC2(f)                                         (dl_gemm_e4m3)
 
-    ``y`` is the layer's output and ``h`` its residual stream; the next layer's
-    first step adds them.  Seven kernels (eight or nine when an input is too
-    large for a GEMM to quantise itself), chained with PDL on one stream.
-    Every step runs in libdl.so; this class only holds buffers."""
+    ``y`` is the layer's output and ``h`` its residual stream (updated in place);
+    the next layer's first step adds them.  Each RMSNorm call is the producer
+    kernel followed by its GEMM: seven kernels at batch 1 (more when an input
+    is too large for a GEMM to quantise itself), all chained with PDL on one
+    stream.  Everything runs in libdl.so; this class only holds buffers."""
 
     def __init__(self, w_qkv, s_qkv, w_o, s_o, w13, s13, w2, s2, g1, g2, *, Hq, Hkv, d, q_scale, M, B, T,
                  eps: float = 1e-5, cluster: int = 8, device="cuda"):
@@ -141,6 +140,7 @@ class FullDecodeLayer:
         self.ws_qkv, self.ws_o, self.ws_13, self.ws_2 = ws(self.D), ws(Hq * d), ws(self.D), ws(self.F)
         self.ws_attn = None
         self.Lcap_hint = None
+        self.h_mid = torch.empty((M, self.D), dtype=torch.int16, device=self.device)  # h1
         self.qkv = torch.empty((M, self.N_qkv), dtype=torch.int16, device=self.device)
         self.attn_out = torch.empty((M, Hq * d), dtype=torch.int16, device=self.device)
         self.a = torch.empty((M, self.D), dtype=torch.int16, device=self.device)
@@ -161,19 +161,16 @@ class FullDecodeLayer:
             n = dl.dl_decode_attn_workspace_bytes(self.B, self.T, self.Hq, self.Hkv, self.d, Lcap, self.cluster)
             self.ws_attn = torch.zeros(n, dtype=torch.uint8, device=self.device)
             self.Lcap_hint = Lcap
-        ready = flags | dl.DL_FLAG_XQ_READY
-        dl.check(dl.dl_add_rmsnorm_quant(x, h, h, self.g1, M, D, self.eps, self.ws_qkv, stream=stream, flags=flags))
-        dl.check(dl.dl_fc_qkv_scale(None, M, D, self.wp["qkv"], self.s["qkv"], self.Hq, self.Hkv, self.d,
-                                    self.q_scale, self.qkv, self.ws_qkv, stream=stream, flags=ready))
+        dl.check(dl.dl_rmsnorm_fc_qkv_scale(x, h, self.h_mid, self.g1, self.eps, M, D, self.wp["qkv"],
+                                            self.s["qkv"], self.Hq, self.Hkv, self.d, self.q_scale, self.qkv,
+                                            self.ws_qkv, stream=stream, flags=flags))
         dl.check(dl.dl_decode_attn(self.qkv, self.N_qkv, self.B, self.T, self.Hq, self.Hkv, self.d, k_cache,
                                    v_cache, Lcap, seq_lens, 1.0, self.cluster, self.attn_out, self.ws_attn,
                                    stream=stream, flags=flags))
         dl.check(dl.dl_gemm_e4m3(self.attn_out, M, self.Hq * self.d, self.wp["o"], self.s["o"], D, self.a,
                                  self.ws_o, stream=stream, flags=flags))
-        dl.check(dl.dl_add_rmsnorm_quant(self.a, h, h, self.g2, M, D, self.eps, self.ws_13, stream=stream,
-                                         flags=flags))
-        dl.check(dl.dl_fc13_swiglu(None, M, D, self.wp["13"], self.s["13"], self.N2, self.f, self.ws_13,
-                                   stream=stream, flags=ready))
+        dl.check(dl.dl_rmsnorm_fc13_swiglu(self.a, self.h_mid, h, self.g2, self.eps, M, D, self.wp["13"],
+                                           self.s["13"], self.N2, self.f, self.ws_13, stream=stream, flags=flags))
         dl.check(dl.dl_gemm_e4m3(self.f, M, self.F, self.wp["2"], self.s["2"], D, self.y, self.ws_2,
                                  stream=stream, flags=flags))
 

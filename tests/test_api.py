@@ -240,7 +240,7 @@ def test_spec_verify_argument_errors():
 
 
 def test_fp8kv_attention_argument_errors():
-    a = dict(q=FAKE, q_token_stride=1024, B=1, T=1, Hq=8, Hkv=2, d=128, k_cache=FAKE, v_cache=FAKE, kv_scale=FAKE,
+    a = dict(q=FAKE, q_token_stride=1024, B=1, T=1, Hq=8, Hkv=2, d=128, k_cache=FAKE, vt_cache=FAKE, kv_scale=FAKE,
              Lcap=256, seq_lens=FAKE, softmax_scale=0.125, cluster_size=8, out=FAKE, ws=FAKE, ws_bytes=256,
              stream=0, flags=0)
     f = dl.dl_decode_attn_fp8kv
@@ -258,3 +258,27 @@ def test_copy_argument_errors():
     assert dl.dl_copy(FAKE, FAKE + 4096, 17, 0, 0) == dl.DL_ERR_ALIGNMENT
     assert dl.dl_copy(FAKE + 8, FAKE + 4096, 16, 0, 0) == dl.DL_ERR_ALIGNMENT
     assert dl.dl_copy(FAKE, FAKE + 16, 64, 0, 0) == dl.DL_ERR_INVALID_ARG  # overlap
+
+
+def test_fp8kv_cache_capacity_must_be_a_multiple_of_16():
+    a = dict(q=FAKE, q_token_stride=1024, B=1, T=1, Hq=8, Hkv=2, d=128, k_cache=FAKE, vt_cache=FAKE, kv_scale=FAKE,
+             Lcap=200 + 4, seq_lens=FAKE, softmax_scale=0.125, cluster_size=8, out=FAKE, ws=FAKE, ws_bytes=256,
+             stream=0, flags=0)
+    assert dl.dl_decode_attn_fp8kv(**a) == dl.DL_ERR_ALIGNMENT
+
+
+def test_fused_rmsnorm_gemm_argument_errors():
+    base = dict(x=FAKE, residual=FAKE + (1 << 24), h_out=FAKE + (2 << 24), gamma=FAKE + (3 << 24), eps=1e-5, M=1,
+                K=512, w_packed=FAKE + (4 << 24), w_scale=FAKE + (5 << 24), N2=512, out=FAKE + (6 << 24),
+                ws=FAKE + (7 << 24), ws_bytes=1 << 20, stream=0, flags=0)
+    f = dl.dl_rmsnorm_fc13_swiglu
+    assert f(**{**base, "h_out": FAKE + (1 << 24) + 512}) == dl.DL_ERR_INVALID_ARG  # partial overlap with residual
+    assert f(**{**base, "h_out": FAKE + 512}) == dl.DL_ERR_INVALID_ARG  # partial overlap with x
+    assert f(**{**base, "gamma": None}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**base, "eps": 0.0}) == dl.DL_ERR_INVALID_ARG
+    assert f(**{**base, "gamma": FAKE + (3 << 24) + 2}) == dl.DL_ERR_ALIGNMENT
+    assert f(**{**base, "N2": 384}) == dl.DL_ERR_UNSUPPORTED
+    q = dict(x=FAKE, residual=None, h_out=None, gamma=FAKE + (3 << 24), eps=1e-5, M=1, K=512, w_packed=FAKE,
+             w_scale=FAKE, Hq=8, Hkv=2, d=64, q_scale=0.125, qkv=FAKE + (6 << 24), ws=FAKE + (7 << 24),
+             ws_bytes=100, stream=0, flags=0)
+    assert dl.dl_rmsnorm_fc_qkv_scale(**q) == dl.DL_ERR_WORKSPACE

@@ -349,3 +349,60 @@ def test_full_layer_chain(name):
     assert np.isfinite(y).all()
     assert helpers.rel_l2(y, y_ref) <= 2e-2, helpers.rel_l2(y, y_ref)
     assert helpers.rel_l2(helpers.bf16_to_f64(host_u16(h)), helpers.bf16_to_f64(h_ref)) <= 1e-2
+
+
+# ------------------------------------- RMSNorm producer + GEMM in one call --
+
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 24])
+@pytest.mark.parametrize("inputs", ["exact", "random"])
+def test_rmsnorm_fused_into_fc13(M, inputs):
+    """dl_rmsnorm_fc13_swiglu (producer kernel + GEMM in one call).  Exact rows:
+    codes identical to the oracle's, element-wise GEMM rule; random rows:
+    relative L2 (a code at a rounding tie may differ)."""
+    K, N2 = 2048, 512
+    g = np.random.default_rng(700 + M + (inputs == "exact") * 50)
+    if inputs == "exact":
+        x = exact_rows(g, M, K)
+        r = x.copy()
+        eps = EPS_EXACT
+    else:
+        x = dg.bf16_normal(g, (M, K))
+        r = dg.bf16_normal(g, (M, K), std=2.0)
+        eps = 1e-5
+    gam = dg.rmsnorm_gain(g, K)
+    w, s_w = dg.e4m3_weight(g, N2, K)
+    wp = torch.empty((N2, K), dtype=torch.uint8, device="cuda")
+    dl.check(dl.dl_pack_fp8_weight(dev_u8(w), wp, N2, K, dl.DL_PACK_SWIGLU))
+    ws, n = new_ws(M, K)
+    hd = torch.full((M, K), -1, dtype=torch.int16, device="cuda")
+    out = torch.empty((M, N2 // 2), dtype=torch.int16, device="cuda")
+    for _ in range(2):  # twice on one stream: the second call must not see the first's h
+        dl.check(dl.dl_rmsnorm_fc13_swiglu(dev_u16(x), dev_u16(r), hd, dev_u16(gam), eps, M, K, wp, dev_f32(s_w), N2,
+                                           out, ws, n))
+    assert dl.dl_read_status(ws) == dl.DL_OK
+    h_ref, _, xq_ref, sx_ref = oracle.add_rmsnorm_quant(x, r, gam, eps)
+    assert np.array_equal(host_u16(hd), h_ref)
+    ref = oracle.fc13_swiglu_q(xq_ref, sx_ref, w, s_w)
+    if inputs == "exact":
+        assert np.array_equal(ws[256:256 + M * K].cpu().numpy().reshape(M, K), xq_ref)
+        helpers.check_gemm(host_u16(out), ref, f"fused norm fc13 M={M}")
+    else:
+        assert helpers.rel_l2(helpers.bf16_to_f64(host_u16(out)), ref) <= helpers.GEMM_REL_L2
+
+
+@pytest.mark.parametrize("M", [1, 5])
+def test_rmsnorm_fused_into_qkv_without_residual_or_h(M):
+    K, Hq, Hkv, d = 1024, 4, 2, 64
+    N = (Hq + 2 * Hkv) * d
+    g = np.random.default_rng(760 + M)
+    x = exact_rows(g, M, K)
+    gam = dg.rmsnorm_gain(g, K)
+    w, s_w = dg.e4m3_weight(g, N, K)
+    ws, n = new_ws(M, K)
+    out = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    dl.check(dl.dl_rmsnorm_fc_qkv_scale(dev_u16(x), None, None, dev_u16(gam), EPS_EXACT, M, K, pack(dev_u8(w), N, K),
+                                        dev_f32(s_w), Hq, Hkv, d, 0.125, out, ws, n))
+    assert dl.dl_read_status(ws) == dl.DL_OK
+    _, _, xq_ref, sx_ref = oracle.add_rmsnorm_quant(x, None, gam, EPS_EXACT)
+    helpers.check_gemm(host_u16(out), oracle.fc_qkv_scale_q(xq_ref, sx_ref, w, s_w, Hq, Hkv, d, 0.125),
+                       f"fused norm qkv M={M}")
