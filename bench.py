@@ -45,6 +45,9 @@ def parse_args():
     p.add_argument("--no-full-layer", action="store_true", help="skip the whole-layer (7-kernel) figure")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="only run this many direct-launch layer steps (for a profiler), print no JSON line")
+    p.add_argument("--profile-moe", type=int, default=0,
+                   help="only run this many grouped MoE FC13 + SwiGLU calls of the moe64 workload (for a "
+                        "profiler), print no JSON line")
     p.add_argument("--profile-next", type=int, default=0,
                    help="only run this many direct-launch whole-layer steps, FP8-cache attention calls and "
                         "verification calls (for a profiler), print no JSON line")
@@ -372,6 +375,32 @@ def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, 
     return out
 
 
+def profile_moe(n, device, experts=16):
+    """n grouped FC13 + SwiGLU calls at the moe64 shapes (64 tokens, experts of
+    [16384, 5120] e4m3 drawn on the device, top-1 uniform routes) over a bank of
+    `experts` experts: 16 (1.3 GB) keeps a multi-pass profiler capture small."""
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200 import dl
+
+    wl = dg.WORKLOADS["moe64"]
+    g = dg.rng(wl.seed)
+    x = torch.from_numpy(dg.bf16_normal(g, (wl.M, wl.K)).view("int16")).to(device)
+    ids = torch.from_numpy(g.integers(0, experts, size=wl.M).astype("int32")).to(device)
+    gen = torch.Generator(device=device).manual_seed(wl.seed)
+    bank = torch.empty((experts, wl.N2, wl.K), dtype=torch.uint8, device=device)
+    scales = torch.empty(experts, dtype=torch.float32, device=device)
+    for e in range(experts):
+        codes, s = dg.e4m3_weight_torch(gen, wl.N2, wl.K, device)
+        dl.check(dl.dl_pack_fp8_weight(codes, bank[e], wl.N2, wl.K, dl.DL_PACK_SWIGLU))
+        scales[e] = s
+    out = torch.empty((wl.M, wl.N2 // 2), dtype=torch.int16, device=device)
+    ws = torch.zeros(dl.dl_workspace_bytes(wl.M, wl.K), dtype=torch.uint8, device=device)
+    for _ in range(n):
+        dl.check(dl.dl_moe_fc13_swiglu_grouped(x, wl.M, wl.K, ids, experts, bank, scales, wl.N2, out, ws))
+    dl.check(dl.dl_read_status(ws))
+
+
 def profile_next_rows(wl, n, seq_lens, device, cluster):
     """n direct-launch steps of the whole layer, n FP8-cache attention calls and
     n verification calls over the full vocabulary, on two replicas (the input of
@@ -440,6 +469,12 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     dl_build.build()
     dl.lib()
+
+    if args.profile_moe > 0:  # the grouped expert GEMM alone, for a profiler
+        profile_moe(args.profile_moe, device)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     wl = dg.WORKLOADS[args.workload]
     cluster = args.cluster or wl.cluster
