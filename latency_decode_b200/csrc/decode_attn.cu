@@ -432,8 +432,11 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   __syncthreads();  // the ring is drained: reuse it for the per-warp states
   pdl_wait();
   const int R = a.R;
-  float* wo = reinterpret_cast<float*>(ring);             // [W][R][D] per-warp o
-  float* wm = wo + kAttnConsumers * R * D;                // [W][R]
+  // Rows of the per-warp o are padded to D + 4 floats: the 4 lanes of a fragment
+  // that write the same column of 4 different rows then hit 4 different banks.
+  constexpr int DP = D + 4;
+  float* wo = reinterpret_cast<float*>(ring);             // [W][R][DP] per-warp o
+  float* wm = wo + kAttnConsumers * R * DP;               // [W][R]
   float* wl = wm + kAttnConsumers * R;                    // [W][R]
   if (warp < kAttnConsumers) {
 #pragma unroll
@@ -448,8 +451,8 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           }
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
-            wo[(warp * R + rho) * D + mt * 16 + g] = o[mt][nt][j];
-            wo[(warp * R + rho) * D + mt * 16 + g + 8] = o[mt][nt][2 + j];
+            wo[(warp * R + rho) * DP + mt * 16 + g] = o[mt][nt][j];
+            wo[(warp * R + rho) * DP + mt * 16 + g + 8] = o[mt][nt][2 + j];
           }
         }
       }
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       const float lw = wl[w * R + rho];
       if (lw > 0.0f) {
         const float f = ex2(wm[w * R + rho] - M);
-        const float4 v = *reinterpret_cast<const float4*>(wo + (w * R + rho) * D + c4 * 4);
+        const float4 v = *reinterpret_cast<const float4*>(wo + (w * R + rho) * DP + c4 * 4);
         acc.x += v.x * f;
         acc.y += v.y * f;
         acc.z += v.z * f;
@@ -659,7 +662,7 @@ struct AttnPlan {
 template <int D, int NT, int W, bool F8>
 static AttnPlan attn_plan(int R, int S) {
   constexpr int STAGE_BYTES = F8 ? 2 * (16 * W) * D : 2 * (D / 64) * (16 * W) * 128;
-  const int merge_bytes = (W * R * D + 2 * W * R) * 4;
+  const int merge_bytes = (W * R * (D + 4) + 2 * W * R) * 4;  // per-warp o rows padded to D + 4
   const int I = R * (D / 4);
   const int Q = (I + S - 1) / S;
   const int recv_bytes = S * Q * (16 + 8);
