@@ -109,6 +109,40 @@ def time_oracle(wl, inp, seconds, min_reps=1, max_reps=10**6):
     return dt / reps * 1e6, reps, dt
 
 
+def _oracle_worker(job):
+    """One host core's share of the all-cores oracle baseline (runs in a spawned
+    process): its own copy of the inputs, one warm-up layer, then whole layers
+    until `seconds` have passed."""
+    name, seconds = job
+    from latency_decode_b200 import datagen as dg
+    wl = dg.WORKLOADS[name]
+    inp = oracle_layer_inputs(wl)
+    oracle_layer(wl, inp)
+    _, reps, dt = time_oracle(wl, inp, seconds, min_reps=1)
+    return reps, dt
+
+
+def host_cores(cap=16):
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(n, cap))
+
+
+def time_oracle_all_cores(wl, seconds, cores):
+    """The single-threaded oracle on `cores` host cores at once, one whole layer
+    per process at a time (independent layers; the oracle itself is unchanged).
+    Returns (us per layer at the aggregate rate, layers timed).  Spawned
+    processes: never forked from a process that holds a CUDA context."""
+    import multiprocessing
+    ctx = multiprocessing.get_context("spawn")
+    with ctx.Pool(cores) as pool:
+        res = pool.map(_oracle_worker, [(wl.name, seconds)] * cores)
+    rate = sum(r / dt for r, dt in res)
+    return 1e6 / rate, sum(r for r, _ in res)
+
+
 def run_reference(args):
     rank = env_int("RANK", 0)
     if rank != 0:
@@ -707,13 +741,19 @@ def run_ours(args):
     h2d = hx.numel() * 2
     d2h = hout.numel() * 2
 
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and not args.no_cpu_baseline:
         inp = oracle_layer_inputs(wl)
         us_cpu, reps, secs = time_oracle(wl, inp, args.cpu_seconds, min_reps=1)
         cpu = {"value": us_cpu, "unit": "us", "cores": 1, "kind": "oracle",
                "sample": f"{reps} full {wl.name} layers ({secs:.1f} s) through the single-threaded FP64 C++ "
                          "oracle on the host"}
+        cores = host_cores()
+        if cores > 1:
+            us_all, reps_all = time_oracle_all_cores(wl, args.cpu_seconds, cores)
+            cpu_all = {"value": us_all, "unit": "us", "cores": cores, "kind": "oracle",
+                       "sample": f"{reps_all} full {wl.name} layers in {args.cpu_seconds:.1f} s, one single-threaded "
+                                 f"oracle process per core on {cores} host cores (independent layers)"}
 
     if world > 1:
         dist.barrier(device_ids=[local])
@@ -741,6 +781,7 @@ def run_ours(args):
         "e2e": {"value": us_e2e, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "mode": e2e_mode, "direct_launch_us": us_e2e_direct},
         "cpu_baseline": cpu,
+        "cpu_baseline_all_cores": cpu_all,
         "gpu_launches": (2 * gl + 1) * args.steps,
         "full_layer": full,
         "next_rows": next_rows,

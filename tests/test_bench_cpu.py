@@ -73,3 +73,14 @@ def test_reference_arm_two_ranks_under_torchrun():
     out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, check=True).stdout
     lines = _json_lines(out)
     assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_oracle_baseline_on_two_host_cores():
+    """The all-cores CPU baseline: two spawned single-threaded oracle processes,
+    each timing whole layers of its own copy of the inputs."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from latency_decode_b200 import datagen as dg
+    us, reps = bench.time_oracle_all_cores(dg.WORKLOADS["tiny"], 0.3, 2)
+    assert us > 0 and reps >= 2
+    assert 1 <= bench.host_cores() <= 16
