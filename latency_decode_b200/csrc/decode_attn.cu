@@ -27,7 +27,8 @@
 //  * merges: the W warp states merge in shared memory; each CTA then pushes
 //    its state of every output item (a float4 of o and the row's (m, l)) into
 //    the receive buffer of the CTA of the cluster that owns the item, through
-//    distributed shared memory; after one cluster barrier each owner merges
+//    distributed shared memory, with non-blocking stores that count their
+//    bytes on the owner's mbarrier; once its bytes are in, each owner merges
 //    the S states (M* = max m_i, L* = sum l_i 2^(m_i-M*), o = sum o_i
 //    2^(m_i-M*) / L*).  With P = 1 that is the final result.  With P > 1 (used
 //    when B*Hkv*S CTAs would leave the GPU half idle) each cluster stores its
@@ -119,11 +120,13 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   uint2* qs = reinterpret_cast<uint2*>(ring + a.stages * STAGE_BYTES);        // [KS][NT][32]
   uint8_t* recv_base = smem + a.recv_off;                                      // DSMEM receive buffer
   uint64_t* bars = reinterpret_cast<uint64_t*>(qs + KS * NT * 32);
-  int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages);
+  // bars: [stages] full, [stages] empty, then the receive barrier of the merge
+  int* abort_word = reinterpret_cast<int*>(bars + 2 * a.stages + 1);
   int* last_word = abort_word + 1;
   volatile int* abort_flag = abort_word;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8u * a.stages;
+  const uint32_t recv_bar = empty0 + 8u * a.stages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -173,11 +176,15 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       mbar_init(full0 + 8u * s, 1);
       mbar_init(empty0 + 8u * s, kAttnConsumers);
     }
+    if (F8) mbar_init(recv_bar, 1);
     *abort_word = 0;
     *last_word = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  // F8: every CTA's receive barrier is initialised before any peer stores into
+  // it (the matching wait comes just before the merge's pushes).
+  if constexpr (F8) cluster_arrive();
 
   const int g = lane >> 2;   // MMA group id (row of the A/C fragments)
   const int q4 = lane & 3;   // thread in group
@@ -463,13 +470,22 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   // Outputs are I = R*D/4 float4 items; CTA c of the cluster owns items
   // [c*Q, (c+1)*Q).  Every CTA stores its state of item i -- the float4 of o
   // and the (m, l) of its row -- straight into the receive buffer of the owner
-  // of i (two remote shared-memory stores per item, no round trip); one
-  // cluster barrier later each owner merges the S states of its items locally.
+  // of i (two remote shared-memory stores per item, no round trip).  bf16
+  // cache: plain remote stores, then one cluster barrier.  FP8 cache:
+  // non-blocking remote stores (st.async) that count their bytes on the
+  // owner's receive barrier, where the owner waits (measured faster for this
+  // variant only).  Each owner then merges the S states of its items locally.
   const int I = R * (D / 4);
   const int Q = (I + S - 1) / S;
+  const int my0 = rank * Q;
+  const int cnt = max(0, min(I, my0 + Q) - my0);
   float4* rv_o = reinterpret_cast<float4*>(recv_base);      // [S][Q]
   float2* rv_ml = reinterpret_cast<float2*>(rv_o + S * Q);  // [S][Q] (m, l)
   const uint32_t rv_o_l = smem_u32(rv_o), rv_ml_l = smem_u32(rv_ml);
+  if constexpr (F8) {
+    cluster_wait();  // every receive barrier of the cluster is initialised
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S * cnt * (16 + 8)));
+  }
   for (int it = threadIdx.x; it < I; it += kAttnThreads) {
     const int rho = it / (D / 4);
     const int c4 = it - rho * (D / 4);
@@ -494,17 +510,26 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     }
     const int owner = it / Q;
     const uint32_t slot_i = static_cast<uint32_t>(rank * Q + (it - owner * Q));
-    dsmem_st_f32x4(dsmem_addr(rv_o_l + 16u * slot_i, owner), acc);
-    dsmem_st_f32x2(dsmem_addr(rv_ml_l + 8u * slot_i, owner), M, lsum);
+    if constexpr (F8) {
+      const uint32_t owner_bar = dsmem_addr(recv_bar, owner);
+      dsmem_st_async_f32x4(dsmem_addr(rv_o_l + 16u * slot_i, owner), acc, owner_bar);
+      dsmem_st_async_f32x2(dsmem_addr(rv_ml_l + 8u * slot_i, owner), M, lsum, owner_bar);
+    } else {
+      dsmem_st_f32x4(dsmem_addr(rv_o_l + 16u * slot_i, owner), acc);
+      dsmem_st_f32x2(dsmem_addr(rv_ml_l + 8u * slot_i, owner), M, lsum);
+    }
   }
-  cluster_sync();  // every state of my items has landed in my receive buffer
+  // every state of my items has landed in my receive buffer
+  if constexpr (F8) {
+    if (!mbar_wait_cluster(recv_bar, 0, budget)) set_status(a.status, kStatusTimeout);
+  } else {
+    cluster_sync();
+  }
 
   // ---- merge the S CTA states of my items ----
   const float out_scale = F8 ? __ldg(a.kv_scale + 1) : 1.0f;  // F8: the cache holds v / s_v
   const long long head = static_cast<long long>(b) * a.Hkv + hk;
   const long long slot = head * a.P + split;
-  const int my0 = rank * Q;
-  const int cnt = max(0, min(I, my0 + Q) - my0);
   for (int k = threadIdx.x; k < cnt; k += kAttnThreads) {
     const int it = my0 + k;
     const int rho = it / (D / 4);
@@ -597,7 +622,8 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
     }
   }
-  // No trailing cluster barrier: after the one above, no CTA touches another CTA's shared memory.
+  // No trailing cluster barrier: once a CTA has received all of its items, no
+  // other CTA touches its shared memory.
 }
 
 // ---- host side ----------------------------------------------------------------------
@@ -668,7 +694,7 @@ static AttnPlan attn_plan(int R, int S) {
   const int recv_bytes = S * Q * (16 + 8);
   const int qs_bytes = (D / 16) * NT * 32 * 8;
   auto smem_for = [&](int st) {
-    return 1024 + st * STAGE_BYTES + qs_bytes + 2 * st * 8 + 16 + recv_bytes + 16;
+    return 1024 + st * STAGE_BYTES + qs_bytes + (2 * st + 1) * 8 + 16 + recv_bytes + 16;
   };
   int stages = D == 128 ? 3 : 6;
   // W = 4 is chosen to put two CTAs on each SM: give up ring depth (down to
@@ -682,7 +708,7 @@ static AttnPlan attn_plan(int R, int S) {
   AttnPlan pl;
   pl.stages = stages;
   pl.smem = smem_for(stages);
-  pl.recv_off = ((stages * STAGE_BYTES + qs_bytes + 2 * stages * 8 + 16) + 15) & ~15;
+  pl.recv_off = ((stages * STAGE_BYTES + qs_bytes + (2 * stages + 1) * 8 + 16) + 15) & ~15;
   return pl;
 }
 
