@@ -231,10 +231,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       const uint64_t pol = l2_policy_evict_first();
       const int n_issue = a.debug ? nsub - 1 : nsub;  // test hook: withhold the last stage
       int issued = 0;
+      // stage s and round parity kept incrementally (no division by the
+      // runtime ring depth on this single-thread issue path)
+      int s = 0;
+      uint32_t round_par = 0;  // (i / stages) & 1
       for (int i = 0; i < n_issue; ++i) {
-        const int s = i % a.stages;
-        if (i >= a.stages &&
-            !mbar_wait(empty0 + 8u * s, static_cast<uint32_t>((i / a.stages) - 1) & 1u, budget, abort_flag)) {
+        if (i >= a.stages && !mbar_wait(empty0 + 8u * s, round_par ^ 1u, budget, abort_flag)) {
           set_status(a.status, kStatusTimeout);
           *abort_flag = 1;
           break;
@@ -243,6 +245,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
         bulk_load(smem_u32(ring + s * kSubBytes), wsrc + static_cast<long long>(i) * kSubBytes, kSubBytes,
                   full0 + 8u * s, pol);
         issued = i + 1;
+        if (++s == a.stages) {
+          s = 0;
+          round_par ^= 1u;
+        }
       }
       if (*abort_flag) {  // let the copies still in flight land before the CTA can exit
         const int first = issued > a.stages ? issued - a.stages : 0;
@@ -260,8 +266,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
         *abort_flag = 1;
       } else {
         const uint32_t idesc = e4m3_idesc(128, npad);
+        int s = 0;
+        uint32_t round_par = 0;  // (i / stages) & 1, kept incrementally like the producer's
         for (int i = 0; i < nsub; ++i) {
-          const int s = i % a.stages;
           const int kbl = i / SUBS;
           const int which = i % SUBS;
           const int bslot = kbl % kBStages;
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
             *abort_flag = 1;
             break;
           }
-          if (!mbar_wait(full0 + 8u * s, static_cast<uint32_t>(i / a.stages) & 1u, budget, abort_flag)) {
+          if (!mbar_wait(full0 + 8u * s, round_par, budget, abort_flag)) {
             set_status(a.status, kStatusTimeout);
             *abort_flag = 1;
             break;
@@ -288,6 +295,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
           ++n_mma;
           tc_commit(empty0 + 8u * s);  // stage free once these MMAs have read it
           if (stream_b && which == SUBS - 1) tc_commit(bempty0 + 8u * bslot);  // B slot free too
+          if (++s == a.stages) {
+            s = 0;
+            round_par ^= 1u;
+          }
         }
       }
       if (n_mma > 0) tc_commit(done);
