@@ -214,10 +214,10 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       const int z = b * a.Hkv + hk;
       const int n_issue = (a.debug && n_tiles > 0) ? n_tiles - 1 : n_tiles;  // test hook
       int issued = 0;
+      int s = 0;               // stage of tile i, and
+      uint32_t round_par = 0;  // (i / stages) & 1, both kept without a division
       for (int i = 0; i < n_issue; ++i) {
-        const int s = i % a.stages;
-        if (i >= a.stages &&
-            !mbar_wait(empty0 + 8u * s, static_cast<uint32_t>((i / a.stages) - 1) & 1u, budget, abort_flag)) {
+        if (i >= a.stages && !mbar_wait(empty0 + 8u * s, round_par ^ 1u, budget, abort_flag)) {
           set_status(a.status, kStatusTimeout);
           *abort_flag = 1;
           break;
@@ -237,6 +237,10 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           }
         }
         issued = i + 1;
+        if (++s == a.stages) {
+          s = 0;
+          round_par ^= 1u;
+        }
       }
       if (*abort_flag) {
         const int first = issued > a.stages ? issued - a.stages : 0;

@@ -307,11 +307,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     __syncwarp();
   } else {
     // ---- activation stager: e4m3 rows -> swizzled K-major B operand ----
-    pdl_wait();  // x (or x_q and s_x) is written by the preceding kernel
-    pdl_trigger();
     const int t = threadIdx.x - 64;
     const int per_row = nkb * 8;  // 16-byte chunks per token row of this K slice
     const int chunks = npad * per_row;
+    // row and chunk-in-row of this thread's first chunk; the loops below step
+    // them by 64 chunks without a division
+    const int row_t = t / per_row;
+    const int rem_t = t - row_t * per_row;
+    pdl_wait();  // x (or x_q and s_x) is written by the preceding kernel
+    pdl_trigger();
     if (a.x != nullptr) {
       // Fused quantiser (A1): amax over the whole [M][K] input, then this CTA's
       // K slice straight into the B operand.  Same arithmetic as act_quant.cu.
@@ -325,18 +329,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       // needs no second trip to memory.
       constexpr int kKeep = 4;
       uint4 keep[2 * kKeep];
+      {
+        int row = row_t, rem = rem_t;
 #pragma unroll
-      for (int j = 0; j < kKeep; ++j) {
-        keep[2 * j] = make_uint4(0u, 0u, 0u, 0u);
-        keep[2 * j + 1] = keep[2 * j];
-        const int c = t + 64 * j;
-        const int row = c / per_row;
-        if (c < chunks && row < n_tok) {
-          const int rem = c - row * per_row;
-          const uint4* src =
-              xv + ((static_cast<long long>(row) * a.K + (kb0 + (rem >> 3)) * 128 + (rem & 7) * 16) >> 3);
-          keep[2 * j] = __ldcg(src);
-          keep[2 * j + 1] = __ldcg(src + 1);
+        for (int j = 0; j < kKeep; ++j) {
+          keep[2 * j] = make_uint4(0u, 0u, 0u, 0u);
+          keep[2 * j + 1] = keep[2 * j];
+          const int c = t + 64 * j;
+          if (c < chunks && row < n_tok) {
+            const uint4* src =
+                xv + ((static_cast<long long>(row) * a.K + (kb0 + (rem >> 3)) * 128 + (rem & 7) * 16) >> 3);
+            keep[2 * j] = __ldcg(src);
+            keep[2 * j + 1] = __ldcg(src + 1);
+          }
+          rem += 64;
+          while (rem >= per_row) {
+            rem -= per_row;
+            ++row;
+          }
         }
       }
       // amax over all of x: 16 independent 16-byte loads in flight per thread per
@@ -362,9 +372,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       if (t == 0) misc->sx = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
       const bool publish = blockIdx.y == 0 && blockIdx.z == 0;  // one CTA column writes x_q / s_x
       if (publish && rank == 0 && t == 0) *a.s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      for (int c = t, j = 0; c < chunks; c += 64, ++j) {
-        const int row = c / per_row;
-        const int rem = c - row * per_row;
+      for (int c = t, j = 0, row = row_t, rem = rem_t; c < chunks; c += 64, ++j) {
         const int kbl = rem >> 3;
         const int ch = rem & 7;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -390,6 +398,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
                                     (kb0 + kbl) * 128 + ch * 16) = v;
         uint8_t* dst = bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = v;
+        rem += 64;
+        while (rem >= per_row) {
+          rem -= per_row;
+          ++row;
+        }
       }
       fence_async_smem();
       mbar_arrive(xready);
@@ -464,11 +477,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       uint32_t r[8];
       tmem_ld_x8(lane_base + static_cast<uint32_t>(c0), r);
       tmem_wait_ld();
+      // npad is a multiple of 8, so the 8 columns share one sub-accumulator
+      const int which = (SUBS == 2 && c0 >= npad) ? 1 : 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int col = c0 + j;
-        const int which = col / npad;
-        const int m = col - which * npad;
+        const int m = c0 - which * npad + j;
         if (m < n_tok)
           dsmem_st_f32(dst + static_cast<uint32_t>((((rank * SUBS + which) * npad + m) * Qr + k) * 4),
                        __uint_as_float(r[j]));
@@ -524,12 +537,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
+        const int cq = c0 + 8 * q;  // 8 columns of one sub-accumulator (npad is a multiple of 8)
+        const int mq = cq - ((SUBS == 2 && cq >= npad) ? npad : 0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = c0 + 8 * q + j;
-          const int m = col % npad;
-          if (col < ncols && m < n_tok) part[col * 128 + row] = __uint_as_float(r[q][j]);
-        }
+        for (int j = 0; j < 8; ++j)
+          if (cq < ncols && mq + j < n_tok) part[(cq + j) * 128 + row] = __uint_as_float(r[q][j]);
       }
     }
   }
