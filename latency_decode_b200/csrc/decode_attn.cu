@@ -65,6 +65,7 @@ struct AttnArgs {
   int lpt;             // 1: grid z visits the sequences longest first
   int P;
   int stages;
+  uint32_t stages_magic;  // ceil(2^32 / stages): i / stages == umulhi(i, magic) for i < 2^32 / stages
   int recv_off;        // byte offset of the DSMEM receive buffer
   int debug;
 };
@@ -297,9 +298,12 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
 
     for (int i = 0; i < n_tiles; ++i) {
-      const int s = i % a.stages;
+      // stage and round of tile i: a multiply-high by the ring depth's
+      // reciprocal instead of a division
+      const uint32_t round = __umulhi(static_cast<uint32_t>(i), a.stages_magic);
+      const int s = i - static_cast<int>(round) * a.stages;
       bool ok = !*abort_flag;
-      if (ok && !mbar_wait(full0 + 8u * s, static_cast<uint32_t>(i / a.stages) & 1u, budget, abort_flag)) {
+      if (ok && !mbar_wait(full0 + 8u * s, round & 1u, budget, abort_flag)) {
         set_status(a.status, kStatusTimeout);
         *abort_flag = 1;
         ok = false;
@@ -808,6 +812,7 @@ static cudaError_t launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, c
   const AttnPlan pl = attn_plan<D, NT, W, F8>(a.R, p.cluster);
   AttnArgs args = a;
   args.stages = pl.stages;
+  args.stages_magic = static_cast<uint32_t>((0x100000000ull + pl.stages - 1) / pl.stages);
   args.recv_off = pl.recv_off;
   cudaError_t e = attn_configure<D, NT, W, F8>(pl, p.cluster);
   if (e != cudaSuccess) return e;
