@@ -84,3 +84,24 @@ def test_oracle_baseline_on_two_host_cores():
     us, reps = bench.time_oracle_all_cores(dg.WORKLOADS["tiny"], 0.3, 2)
     assert us > 0 and reps >= 2
     assert 1 <= bench.host_cores() <= 16
+
+
+def test_recorded_traffic_matches_the_current_source_only(tmp_path, monkeypatch):
+    """The bench's ncu traffic record: found for the committed FC13 capture, and
+    ignored once the recorded source digest no longer matches the file."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.recorded_traffic("gemm_e4m3_kernel<1>", "layer_b1") is not None
+    assert bench.recorded_traffic("gemm_e4m3_kernel<1>", "no_such_workload") is None
+    # a copy of the tree layout whose record carries a stale digest
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "src.cu").write_text("// kernel source\n")
+    (tmp_path / "profiles" / "k.md").write_text(
+        "traffic-record: kernel=k workload=w bytes_per_launch=123 source=src.cu sha256_16=0000000000000000\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k", "w") is None
+    import hashlib
+    digest = hashlib.sha256(b"// kernel source\n").hexdigest()[:16]
+    (tmp_path / "profiles" / "k.md").write_text(
+        f"traffic-record: kernel=k workload=w bytes_per_launch=123 source=src.cu sha256_16={digest}\n")
+    assert bench.recorded_traffic("k", "w") == 123
