@@ -742,7 +742,7 @@ def run_ours(args):
     d2h = hout.numel() * 2
 
     cpu = cpu_all = None
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the CPU baseline is an N = 1 figure
         inp = oracle_layer_inputs(wl)
         us_cpu, reps, secs = time_oracle(wl, inp, args.cpu_seconds, min_reps=1)
         cpu = {"value": us_cpu, "unit": "us", "cores": 1, "kind": "oracle",
