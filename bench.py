@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 METRIC = "µs per decode layer; achieved HBM TB/s vs B200 peak (FP8 GEMM, split-KV attn)"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse_args():
@@ -43,6 +44,8 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline sample length")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-full-layer", action="store_true", help="skip the whole-layer (7-kernel) figure")
+    p.add_argument("--configs", default="verify4,batch16x4,moe64",
+                   help="other workloads measured after the headline (comma list, or 'none')")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="only run this many direct-launch layer steps (for a profiler), print no JSON line")
     p.add_argument("--profile-moe", type=int, default=0,
@@ -89,15 +92,17 @@ def oracle_layer_inputs(wl):
 
 
 def oracle_layer(wl, inp):
-    """One layer through the CPU oracle (same steps as the GPU path)."""
+    """One layer through the CPU oracle (same steps as the GPU path).  Returns
+    (qkv, attention output, FC13 output), float64."""
     import numpy as np
     import oracle
     from latency_decode_b200 import datagen as dg
     qkv = oracle.fc_qkv_scale(inp["x1"], inp["w_qkv"], inp["s_qkv"], wl.Hq, wl.Hkv, wl.d, inp["q_scale"])
     qb = dg.bf16_bits(qkv.astype(np.float32))
-    oracle.decode_attn(qb.ravel(), wl.n_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, inp["k_cache"], inp["v_cache"],
-                       inp["seq_lens"], 1.0)
-    oracle.fc13_swiglu(inp["x2"], inp["w13"], inp["s13"])
+    attn = oracle.decode_attn(qb.ravel(), wl.n_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, inp["k_cache"],
+                              inp["v_cache"], inp["seq_lens"], 1.0)
+    ffn = oracle.fc13_swiglu(inp["x2"], inp["w13"], inp["s13"])
+    return qkv, attn, ffn
 
 
 def time_oracle(wl, inp, seconds, min_reps=1, max_reps=10**6):
@@ -109,19 +114,6 @@ def time_oracle(wl, inp, seconds, min_reps=1, max_reps=10**6):
     return dt / reps * 1e6, reps, dt
 
 
-def _oracle_worker(job):
-    """One host core's share of the all-cores oracle baseline (runs in a spawned
-    process): its own copy of the inputs, one warm-up layer, then whole layers
-    until `seconds` have passed."""
-    name, seconds = job
-    from latency_decode_b200 import datagen as dg
-    wl = dg.WORKLOADS[name]
-    inp = oracle_layer_inputs(wl)
-    oracle_layer(wl, inp)
-    _, reps, dt = time_oracle(wl, inp, seconds, min_reps=1)
-    return reps, dt
-
-
 def host_cores(cap=16):
     try:
         n = len(os.sched_getaffinity(0))
@@ -130,17 +122,80 @@ def host_cores(cap=16):
     return max(1, min(n, cap))
 
 
-def time_oracle_all_cores(wl, seconds, cores):
-    """The single-threaded oracle on `cores` host cores at once, one whole layer
-    per process at a time (independent layers; the oracle itself is unchanged).
-    Returns (us per layer at the aggregate rate, layers timed).  Spawned
-    processes: never forked from a process that holds a CUDA context."""
-    import multiprocessing
-    ctx = multiprocessing.get_context("spawn")
-    with ctx.Pool(cores) as pool:
-        res = pool.map(_oracle_worker, [(wl.name, seconds)] * cores)
-    rate = sum(r / dt for r, dt in res)
-    return 1e6 / rate, sum(r for r, _ in res)
+def sliced_oracle_inputs(wl, inp, fc13_cols=256):
+    """The slices of one layer's inputs that oracle_layer_sliced hands to its
+    threads: the QKV weight rows of each head, the FC13 gate and up rows of each
+    range of `fc13_cols` output columns (gate rows then the matching up rows),
+    and the K and V caches of each kv head.  Built once, outside any timing."""
+    import numpy as np
+    d, F = wl.d, wl.N2 // 2
+    heads = [(c0, c0 + d) for c0 in range(0, wl.n_qkv, d)]
+    w_heads = [np.ascontiguousarray(inp["w_qkv"][c0:c1]) for c0, c1 in heads]
+    cols = [(j0, min(F, j0 + fc13_cols)) for j0 in range(0, F, fc13_cols)]
+    w13 = [np.ascontiguousarray(np.concatenate([inp["w13"][j0:j1], inp["w13"][F + j0:F + j1]])) for j0, j1 in cols]
+    kv = [(np.ascontiguousarray(inp["k_cache"][:, hk:hk + 1]), np.ascontiguousarray(inp["v_cache"][:, hk:hk + 1]))
+          for hk in range(wl.Hkv)]
+    return {"heads": heads, "w_heads": w_heads, "cols": cols, "w13": w13, "kv": kv}
+
+
+def oracle_layer_sliced(wl, inp, sl, pool):
+    """One layer through the CPU oracle with its independent outputs spread over
+    the threads of `pool`: FC_QKV one head of output columns per task, the
+    attention one query head per task, FC13 one range of output columns per
+    task (FC13 runs beside QKV and attention: its input does not depend on
+    them).  Every task is a call of the oracle's own function on a slice of the
+    weights, or on one head, and the tasks fill disjoint parts of the outputs,
+    so the result equals oracle_layer's bit for bit.  ctypes releases the GIL
+    for the duration of each call, so the tasks run on as many host cores as
+    the pool has threads.  Returns (qkv, attention output, FC13 output)."""
+    import numpy as np
+    import oracle
+    from latency_decode_b200 import datagen as dg
+    d, Hq, Hkv = wl.d, wl.Hq, wl.Hkv
+    G = Hq // Hkv
+    qkv = np.zeros((wl.M, wl.n_qkv))
+    ffn = np.zeros((wl.M, wl.N2 // 2))
+    attn = np.zeros((wl.B, wl.T, Hq, d))
+
+    def qkv_task(i):
+        c0, c1 = sl["heads"][i]
+        if c0 < Hq * d:  # one query head: scaled columns
+            qkv[:, c0:c1] = oracle.fc_qkv_scale(inp["x1"], sl["w_heads"][i], inp["s_qkv"], 1, 0, d, inp["q_scale"])
+        else:            # one K or V head: plain columns
+            qkv[:, c0:c1] = oracle.linear(inp["x1"], sl["w_heads"][i], inp["s_qkv"])
+
+    def fc13_task(i):
+        j0, j1 = sl["cols"][i]
+        ffn[:, j0:j1] = oracle.fc13_swiglu(inp["x2"], sl["w13"][i], inp["s13"])
+
+    def attn_task(h, qb):
+        kc, vc = sl["kv"][h // G]
+        attn[:, :, h:h + 1] = oracle.decode_attn(qb[h * d:], wl.n_qkv, wl.B, wl.T, 1, 1, d, kc, vc,
+                                                 inp["seq_lens"], 1.0)
+
+    f13 = [pool.submit(fc13_task, i) for i in range(len(sl["cols"]))]
+    for f in [pool.submit(qkv_task, i) for i in range(len(sl["heads"]))]:
+        f.result()
+    qb = dg.bf16_bits(qkv.astype(np.float32)).ravel()
+    for f in [pool.submit(attn_task, h, qb) for h in range(Hq)] + f13:
+        f.result()
+    return qkv, attn, ffn
+
+
+def time_oracle_threads(wl, inp, seconds, cores, min_reps=1):
+    """Per-layer latency of the oracle with each layer's outputs spread over
+    `cores` host threads (oracle_layer_sliced).  Returns (us per layer, layers
+    timed, seconds)."""
+    from concurrent.futures import ThreadPoolExecutor
+    sl = sliced_oracle_inputs(wl, inp)
+    with ThreadPoolExecutor(max_workers=cores) as pool:
+        oracle_layer_sliced(wl, inp, sl, pool)  # warm-up
+        reps, t0 = 0, time.perf_counter()
+        while reps < min_reps or time.perf_counter() - t0 < seconds:
+            oracle_layer_sliced(wl, inp, sl, pool)
+            reps += 1
+        dt = time.perf_counter() - t0
+    return dt / reps * 1e6, reps, dt
 
 
 def run_reference(args):
@@ -327,27 +382,22 @@ def make_full_layers(wl, R, seed_base, device, cluster):
     return out
 
 
-def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, capture_fn, graph_steps_fn, peak):
+def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, per_call_us, peak):
     """Per-call device time of the rows beyond the headline chain, each timed the
     way the headline kernels are (graphs of back-to-back calls over more than
-    3x L2 of distinct inputs), with its algorithmic bytes and roofline fraction."""
+    3x L2 of distinct inputs, exactly `steps` calls), with its algorithmic bytes
+    and roofline fraction."""
     import torch
     from latency_decode_b200 import dl
 
     out = {}
     RF = len(fl)
 
-    def timed_call(fn, reps):
-        for i in range(3):
-            fn(i)
-        gbig = capture_fn(fn, range(reps))
-        graph_steps_fn(2 * reps, gbig, [gbig], reps)
-        n = max(reps, (steps // reps) * reps)
-        return timed_graph_fn(n, gbig, [gbig], reps) * 1e3 / n
-
-    def entry(us, nbytes, extra=None):
+    def entry(res, nbytes, extra=None):
+        us, mode, lengths = res
         gbs = nbytes / (us * 1e-6) / 1e9
-        e = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak}
+        e = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak, "mode": mode,
+             "graph_steps": lengths}
         e.update(extra or {})
         return e
 
@@ -364,9 +414,9 @@ def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, 
     def norm(i):
         lay, kc, vc, x, hres = fl[i % RF]
         dl.check(dl.dl_add_rmsnorm_quant(x, hres, hres, lay.g1, wl.M, wl.K, 1e-5, lay.ws_qkv, stream=h()))
-    out["o_proj"] = entry(timed_call(o_proj, G), wl.K * wl.k_o)
-    out["fc2"] = entry(timed_call(fc2, G), wl.K * wl.k_fc2)
-    out["add_rmsnorm_quant"] = entry(timed_call(norm, G), 3 * wl.M * wl.K * 2 + wl.M * wl.K,
+    out["o_proj"] = entry(per_call_us(o_proj, G, steps), wl.K * wl.k_o)
+    out["fc2"] = entry(per_call_us(fc2, G, steps), wl.K * wl.k_fc2)
+    out["add_rmsnorm_quant"] = entry(per_call_us(norm, G, steps), 3 * wl.M * wl.K * 2 + wl.M * wl.K,
                                      {"note": "latency-bound at this size"})
     # NEXT-3: attention over an e4m3 cache (half the bytes of the bf16 cache)
     if wl.d == 128:
@@ -386,7 +436,7 @@ def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, 
             dl.check(dl.dl_decode_attn_fp8kv(lay.qkv, lay.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, caches[r][0],
                                              caches[r][1], scales, wl.Lcap, seq_lens, 1.0, cluster, lay.attn_out,
                                              wss[r], stream=h()))
-        out["decode_attn_fp8kv"] = entry(timed_call(attn8, R8 * max(1, 24 // R8)), kv8)
+        out["decode_attn_fp8kv"] = entry(per_call_us(attn8, R8 * max(1, 24 // R8), steps), kv8)
         for w in wss:
             dl.check(dl.dl_read_status(w))
         del caches, wss
@@ -402,7 +452,7 @@ def measure_next_rows(wl, fl, seq_lens, device, cluster, steps, timed_graph_fn, 
     em = torch.empty((wl.B, wl.T), dtype=torch.int32, device=device)
     def verify(i):
         dl.check(dl.dl_spec_verify_greedy(lg[i % RV], wl.B, wl.T, V, dr, tid, nacc, em, None, stream=h()))
-    out["spec_verify_greedy"] = entry(timed_call(verify, RV * max(1, 24 // RV) if RV < 24 else RV), per,
+    out["spec_verify_greedy"] = entry(per_call_us(verify, RV * max(1, 24 // RV) if RV < 24 else RV, steps), per,
                                       {"vocab": V})
     del lg
     torch.cuda.empty_cache()
@@ -474,6 +524,45 @@ def gemm_launches(M, K):
     return 1 if M * K <= 32768 else 2
 
 
+def replay_plan(n: int, period: int) -> list:
+    """Lengths of the CUDA graphs replayed, in order, to run exactly n steps:
+    graphs of `period` PDL-chained steps, then one graph of the remaining
+    n mod period steps.  Every replayed graph chains several steps (a run of
+    fewer than `period` steps is one graph of n steps), so the timed region
+    has the same shape whatever n is; `period` is a multiple of the replica
+    count, so each graph starts again at replica 0."""
+    if n <= 0:
+        return []
+    q, rem = divmod(n, period)
+    return [period] * q + ([rem] if rem else [])
+
+
+class GraphReplayer:
+    """CUDA graphs of fn(0), fn(1), ... fn(L-1) for each length L that
+    replay_plan asks for, captured once; run(n) replays exactly n steps."""
+
+    def __init__(self, fn, period, capture):
+        self.fn, self.period, self.capture = fn, period, capture
+        self.graphs = {}
+
+    def prepare(self, n):
+        for length in sorted(set(replay_plan(n, self.period))):
+            if length not in self.graphs:
+                self.graphs[length] = self.capture(self.fn, range(length))
+        return self
+
+    def run(self, n):
+        self.prepare(n)
+        for length in replay_plan(n, self.period):
+            self.graphs[length].replay()
+
+    def lengths(self, n):
+        return sorted(set(replay_plan(n, self.period)), reverse=True)
+
+    def release(self):
+        self.graphs.clear()
+
+
 def timed(fn, steps, stream):
     import torch
     start = torch.cuda.Event(enable_timing=True)
@@ -485,6 +574,135 @@ def timed(fn, steps, stream):
     end.record(stream)
     torch.cuda.synchronize()
     return start.elapsed_time(end)  # ms
+
+
+def peak_bf16_tflops():
+    """Dense bf16 tensor peak (TFLOP/s): the measured burst figure when the
+    generated file exists, else the recorded fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def measure_dense_config(name, steps, device, rank, per_call_us, peak, peak_bf16):
+    """Chain and per-call figures of one more dense workload (verify4,
+    batch16x4): its own layer copies (> 3x L2 per rotation), the chain
+    FC_QKV -> attention -> FC13 replayed from CUDA graphs, and each kernel
+    family per call, with algorithmic bytes, the fraction of the HBM peak and
+    the tensor-core rate (FP8 GEMMs against twice the bf16 peak, the nominal
+    ratio; bf16 attention against the bf16 peak)."""
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200 import dl
+
+    wl = dg.WORKLOADS[name]
+    cluster = wl.cluster
+    per_layer = wl.n_qkv * wl.K + wl.N2 * wl.K + 2 * wl.B * wl.Hkv * wl.Lcap * wl.d * 2
+    R = max(2, math.ceil(3 * L2_BYTES / per_layer))
+    layers, kvs, xs, seq_lens, sl = make_layers(wl, R, 3000 * (rank + 1) + 100 * wl.seed, device, cluster)
+    h = lambda: torch.cuda.current_stream().cuda_stream
+
+    def step(i):
+        r = i % R
+        layers[r].step(xs[r][0], xs[r][1], kvs[r][0], kvs[r][1], seq_lens, stream=h())
+
+    def call_qkv(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_fc_qkv_scale(xs[r][0], wl.M, wl.K, L_.wp_qkv, L_.s_qkv, wl.Hq, wl.Hkv, wl.d, L_.q_scale,
+                                    L_.qkv, L_.ws_qkv, stream=h()))
+
+    def call_attn(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_decode_attn(L_.qkv, L_.N_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, kvs[r][0], kvs[r][1],
+                                   wl.Lcap, seq_lens, 1.0, cluster, L_.attn_out, L_.ws_attn, stream=h()))
+
+    def call_fc13(i):
+        r = i % R
+        L_ = layers[r]
+        dl.check(dl.dl_fc13_swiglu(xs[r][1], wl.M, wl.K, L_.wp_13, L_.s_13, wl.N2, L_.ffn_out, L_.ws_13,
+                                   stream=h()))
+
+    G = R * max(1, 24 // R)
+    for i in range(3):
+        step(i)
+    chain_us, chain_mode, lengths = per_call_us(step, G, steps)
+    kv_bytes = int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
+    attn_flops = float(sum(4 * wl.Hq * wl.T * int(L) * wl.d for L in sl))  # QK^T and PV, every key of every row
+    fam = {"fc_qkv_scale": (call_qkv, wl.n_qkv * wl.K, 2.0 * wl.M * wl.n_qkv * wl.K, 2 * peak_bf16),
+           "decode_attn": (call_attn, kv_bytes, attn_flops, peak_bf16),
+           "fc13_swiglu": (call_fc13, wl.N2 * wl.K, 2.0 * wl.M * wl.N2 * wl.K, 2 * peak_bf16)}
+    kernels = {}
+    for kname, (fn, nbytes, flops, tpeak) in fam.items():
+        for i in range(3):
+            fn(i)
+        us, mode, _ = per_call_us(fn, G, steps)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        kernels[kname] = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak,
+                          "tensor_tflops": flops / (us * 1e-6) / 1e12,
+                          "tensor_frac": flops / (us * 1e-6) / 1e12 / tpeak, "mode": mode}
+    for lay in layers:
+        lay.read_status(h())
+    layer_bytes = wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes
+    out = {"workload": f"{wl.name}: M={wl.M} B={wl.B} T={wl.T} L={'U[1024,16384]' if wl.L == 0 else wl.L} "
+                       f"cluster={cluster}",
+           "chain_us": chain_us, "alg_bytes": layer_bytes, "achieved_gbs": layer_bytes / (chain_us * 1e-6) / 1e9,
+           "frac": layer_bytes / (chain_us * 1e-6) / 1e9 / peak, "mode": chain_mode, "graph_steps": lengths,
+           "replicas": R, "kernels": kernels}
+    del layers, kvs, xs
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_moe_config(steps, device, per_call_us, peak, peak_bf16):
+    """Grouped MoE FC13 + SwiGLU at the moe64 shapes: 64 tokens routed top-1
+    uniformly (seeded) over 128 experts of [16384, 5120] e4m3 drawn on the
+    device (10.7 GB); each call reads only the touched experts (> 4 GB, far
+    beyond L2)."""
+    import numpy as np
+    import torch
+    from latency_decode_b200 import datagen as dg
+    from latency_decode_b200 import dl
+
+    wl = dg.WORKLOADS["moe64"]
+    g = dg.rng(wl.seed)
+    x = torch.from_numpy(dg.bf16_normal(g, (wl.M, wl.K)).view("int16")).to(device)
+    ids_h = dg.expert_ids_for(wl, g)
+    ids = torch.from_numpy(ids_h).to(device)
+    gen = torch.Generator(device=device).manual_seed(wl.seed)
+    bank = torch.empty((wl.experts, wl.N2, wl.K), dtype=torch.uint8, device=device)
+    scales = torch.empty(wl.experts, dtype=torch.float32, device=device)
+    for e in range(wl.experts):
+        codes, s = dg.e4m3_weight_torch(gen, wl.N2, wl.K, device)
+        dl.check(dl.dl_pack_fp8_weight(codes, bank[e], wl.N2, wl.K, dl.DL_PACK_SWIGLU))
+        scales[e] = s
+        del codes
+    out = torch.empty((wl.M, wl.N2 // 2), dtype=torch.int16, device=device)
+    ws = torch.zeros(dl.dl_workspace_bytes(wl.M, wl.K), dtype=torch.uint8, device=device)
+
+    def call(i):
+        dl.check(dl.dl_moe_fc13_swiglu_grouped(x, wl.M, wl.K, ids, wl.experts, bank, scales, wl.N2, out, ws,
+                                               stream=torch.cuda.current_stream().cuda_stream))
+
+    for i in range(3):
+        call(i)
+    us, mode, lengths = per_call_us(call, 8, steps)
+    dl.check(dl.dl_read_status(ws))
+    touched = int(np.unique(ids_h).size)
+    nbytes = touched * wl.N2 * wl.K
+    flops = 2.0 * wl.M * wl.N2 * wl.K
+    gbs = nbytes / (us * 1e-6) / 1e9
+    res = {"workload": f"moe64: T={wl.M} E={wl.experts} top-1, FC13 {wl.K}->{wl.N2} per expert",
+           "us_per_call": us, "touched_experts": touched, "alg_bytes": nbytes, "achieved_gbs": gbs,
+           "frac": gbs / peak, "tensor_tflops": flops / (us * 1e-6) / 1e12,
+           "tensor_frac": flops / (us * 1e-6) / 1e12 / (2 * peak_bf16), "mode": mode, "graph_steps": lengths}
+    del bank, x, out, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args):
@@ -558,50 +776,60 @@ def run_ours(args):
                 fn(i)
         return g
 
-    G = R * max(1, 24 // R)
-    graphs = None
-    try:
-        graphs = (capture(step, range(G)), [capture(step, [r]) for r in range(R)])
-    except Exception as exc:  # capture refused: fall back to direct launches, and say so
-        graphs = None
-        graph_error = repr(exc)[:200]
-    torch.cuda.synchronize()
-
-    def graph_steps(n, big, singles, period):
-        q, rem = divmod(n, period)
-        for _ in range(q):
-            big.replay()
-        for j in range(rem):
-            singles[(q * period + j) % len(singles)].replay()
-
-    def timed_graph(n, big, singles, period):
+    def timed_replay(rp, n):
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         start.record()
-        graph_steps(n, big, singles, period)
+        rp.run(n)
         end.record()
         torch.cuda.synchronize()
         return start.elapsed_time(end)
 
-    if graphs is not None:
+    def per_call_us(fn, period, n):
+        """Device time per call of exactly n calls fn(0..n-1), replayed from CUDA
+        graphs of `period` chained calls (the same plan as the headline), or
+        launched directly when capture fails.  Returns (us, mode, graph lengths)."""
+        try:
+            rp = GraphReplayer(fn, period, capture).prepare(n)
+            rp.run(n)  # untimed: the same graphs once through
+            us = timed_replay(rp, n) * 1e3 / n
+            lengths = rp.lengths(n)
+            rp.release()
+            return us, "graph", lengths
+        except Exception:
+            return timed(fn, n, torch.cuda.current_stream()) * 1e3 / n, "direct", []
+
+    G = R * max(1, 24 // R)
+    main_rp, graph_error = None, None
+    try:
+        main_rp = GraphReplayer(step, G, capture).prepare(args.steps)
         for _ in range(2):
-            graph_steps(max(args.warmup, 3), graphs[0], graphs[1], G)
+            main_rp.run(args.steps)  # untimed warm-up replays of the timed graphs
+    except Exception as exc:  # capture refused: fall back to direct launches, and say so
+        main_rp = None
+        graph_error = repr(exc)[:200]
+    torch.cuda.synchronize()
 
     # ---- timed region: exactly K whole-layer steps ----
     clocks = ClockSampler(local)
     barrier()
     clocks.start()
-    if graphs is not None:
-        ms = timed_graph(args.steps, graphs[0], graphs[1], G)
-        launch_mode = f"CUDA graph of {G} PDL-chained layer steps, replayed"
+    if main_rp is not None:
+        ms = timed_replay(main_rp, args.steps)
+        graph_lengths = main_rp.lengths(args.steps)
+        launch_mode = (f"CUDA graphs of {' and '.join(map(str, graph_lengths))} PDL-chained layer steps, replayed "
+                       f"({len(replay_plan(args.steps, G))} replays for {args.steps} steps)")
     else:
         ms = timed(step, args.steps, stream)
+        graph_lengths = []
         launch_mode = "direct launches (graph capture failed: " + graph_error + ")"
     barrier()
     clk = clocks.stop()
     for lay in layers:
         lay.read_status(h)
+    if main_rp is not None:
+        main_rp.release()
     us_layer = max_over_ranks(ms * 1e3 / args.steps)
     layer_bytes = wl.n_qkv * wl.K + wl.N2 * wl.K + int(sum(2 * wl.Hkv * int(L) * wl.d * 2 for L in sl))
     if layer_bytes / (us_layer * 1e-6) / 1e9 > 1.2 * peak_hbm()[0]:
@@ -644,21 +872,15 @@ def run_ours(args):
         "decode_attn": (call_attn, kv_bytes, 1),
     }
     peak, peak_kind = peak_hbm()
+    peak_bf16, peak_bf16_kind = peak_bf16_tflops()
     kernels = {}
     for name, (fn, nbytes, launches) in fam.items():
         for i in range(3):
             fn(i)
-        mode = "direct"
-        try:
-            gbig, gs = capture(fn, range(G)), [capture(fn, [r]) for r in range(R)]
-            graph_steps(6, gbig, gs, G)
-            us = timed_graph(args.steps, gbig, gs, G) * 1e3 / args.steps
-            mode = "graph"
-        except Exception:
-            us = timed(fn, args.steps, stream) * 1e3 / args.steps
+        us, mode, lengths = per_call_us(fn, G, args.steps)
         gbs = nbytes / (us * 1e-6) / 1e9
         kernels[name] = {"us_per_call": us, "alg_bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peak,
-                         "launches_per_call": launches, "mode": mode}
+                         "launches_per_call": launches, "mode": mode, "graph_steps": lengths}
     for lay in layers:
         lay.read_status(h)
 
@@ -676,16 +898,7 @@ def run_ours(args):
 
         for i in range(3):
             full_step(i)
-        GF = RF * max(1, 24 // RF)
-        fmode = "direct"
-        try:
-            gbig, gs = capture(full_step, range(GF)), [capture(full_step, [r]) for r in range(RF)]
-            graph_steps(6, gbig, gs, GF)
-            us_full = timed_graph(args.steps, gbig, gs, GF) * 1e3 / args.steps
-            fmode = "graph"
-            del gbig, gs
-        except Exception:
-            us_full = timed(full_step, args.steps, stream) * 1e3 / args.steps
+        us_full, fmode, flengths = per_call_us(full_step, RF * max(1, 24 // RF), args.steps)
         for entry in fl:
             entry[0].read_status(h)
         us_full = max_over_ranks(us_full)
@@ -694,11 +907,10 @@ def run_ours(args):
         full = {"us": us_full, "alg_bytes": fbytes + kv_bytes,
                 "achieved_gbs": (fbytes + kv_bytes) / (us_full * 1e-6) / 1e9,
                 "frac": (fbytes + kv_bytes) / (us_full * 1e-6) / 1e9 / peak,
-                "launches_per_step": f_launches, "mode": fmode, "replicas": RF,
+                "launches_per_step": f_launches, "mode": fmode, "graph_steps": flengths, "replicas": RF,
                 "steps": "add+RMSNorm+quant -> FC_QKV -> attention -> O_proj -> add+RMSNorm+quant -> FC13+SwiGLU "
                          "-> FC2"}
-        next_rows = measure_next_rows(wl, fl, seq_lens, device, cluster, args.steps, timed_graph, capture,
-                                      graph_steps, peak)
+        next_rows = measure_next_rows(wl, fl, seq_lens, device, cluster, args.steps, per_call_us, peak)
         del fl
         torch.cuda.empty_cache()
 
@@ -723,23 +935,35 @@ def run_ours(args):
     # CUDA graphs, one PDL chain.  DecodeLayer.step_host moves the activations
     # in from pinned host memory and the results out with copy kernels, so the
     # chain is not broken by copy nodes.
-    e2e_mode = "direct"
-    us_e2e = us_e2e_direct
-    try:
-        def e2e_graph_step(i):
-            r = i % R
-            layers[r].step_host(hx, hout, kvs[r][0], kvs[r][1], seq_lens,
-                                stream=torch.cuda.current_stream().cuda_stream)
+    def e2e_graph_step(i):
+        r = i % R
+        layers[r].step_host(hx, hout, kvs[r][0], kvs[r][1], seq_lens,
+                            stream=torch.cuda.current_stream().cuda_stream)
 
-        ge_big, ge_single = capture(e2e_graph_step, range(G)), [capture(e2e_graph_step, [r]) for r in range(R)]
-        graph_steps(2 * G, ge_big, ge_single, G)
-        us_e2e = max_over_ranks(timed_graph(args.steps, ge_big, ge_single, G) * 1e3 / args.steps)
-        e2e_mode = f"CUDA graph of {G} steps, each: copy kernel host->device, the chain, copy kernel device->host"
-        del ge_big, ge_single
-    except Exception as exc:
-        e2e_mode = "direct (graph capture failed: " + repr(exc)[:120] + ")"
+    for i in range(3):
+        e2e_graph_step(i)
+    us_e2e, e2e_kind, e2e_lengths = per_call_us(e2e_graph_step, G, args.steps)
+    us_e2e = max_over_ranks(us_e2e)
+    if e2e_kind == "graph":
+        e2e_mode = (f"CUDA graphs of {' and '.join(map(str, e2e_lengths))} steps, each: copy kernel host->device, "
+                    "the chain, copy kernel device->host")
+    else:
+        e2e_mode = "direct (graph capture failed)"
     h2d = hx.numel() * 2
     d2h = hout.numel() * 2
+    for lay in layers:
+        lay.read_status(h)
+    del layers, kvs, xs, dx
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads: per-config chain and kernel figures ----
+    configs = {}
+    names = [] if args.configs == "none" else [c for c in args.configs.split(",") if c and c != wl.name]
+    for name in names:
+        if name == "moe64":
+            configs[name] = measure_moe_config(args.steps, device, per_call_us, peak, peak_bf16)
+        else:
+            configs[name] = measure_dense_config(name, args.steps, device, rank, per_call_us, peak, peak_bf16)
 
     cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the CPU baseline is an N = 1 figure
@@ -750,10 +974,11 @@ def run_ours(args):
                          "oracle on the host"}
         cores = host_cores()
         if cores > 1:
-            us_all, reps_all = time_oracle_all_cores(wl, args.cpu_seconds, cores)
+            us_all, reps_all, secs_all = time_oracle_threads(wl, inp, args.cpu_seconds, cores)
             cpu_all = {"value": us_all, "unit": "us", "cores": cores, "kind": "oracle",
-                       "sample": f"{reps_all} full {wl.name} layers in {args.cpu_seconds:.1f} s, one single-threaded "
-                                 f"oracle process per core on {cores} host cores (independent layers)"}
+                       "sample": f"{reps_all} full {wl.name} layers ({secs_all:.1f} s), one at a time, each "
+                                 f"layer's output columns and query heads spread over {cores} host threads "
+                                 "(per-layer latency; the oracle's own functions on slices)"}
 
     if world > 1:
         dist.barrier(device_ids=[local])
@@ -772,6 +997,7 @@ def run_ours(args):
                      "traffic": recorded_traffic("gemm_e4m3_kernel<1>", wl.name),
                      "alg_bytes_per_launch": wl.N2 * wl.K},
         "kernels": kernels,
+        "graph_steps": graph_lengths,
         "layer_us_direct_launch": us_layer_direct,
         "layer_us_direct_no_pdl": us_layer_nopdl,
         "host_us_per_step_direct": host_us,
@@ -785,6 +1011,8 @@ def run_ours(args):
         "gpu_launches": (2 * gl + 1) * args.steps,
         "full_layer": full,
         "next_rows": next_rows,
+        "configs": configs,
+        "peak_bf16_tflops": {"value": peak_bf16, "kind": peak_bf16_kind},
         "clocks": clk,
         "replicas": R,
     }

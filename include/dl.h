@@ -71,7 +71,10 @@ typedef enum dl_status {
 #define DL_FLAG_PDL 1u            /* launch with Programmatic Dependent Launch */
 #define DL_FLAG_DEBUG_TIMEOUT 2u  /* test hook: shortens every bounded wait to ~2 ms and
                                      withholds the last pipeline load, so the consumer's
-                                     wait runs out and DL_ERR_TIMEOUT is reported */
+                                     wait runs out and DL_ERR_TIMEOUT is reported; in the
+                                     FP8-cache attention merge each owner CTA also expects
+                                     16 bytes more than its peers send, so its receive
+                                     wait runs out as well */
 #define DL_FLAG_XQ_READY 4u        /* GEMM entry points: the workspace already holds x_q and
                                      s_x, written into this same workspace by
                                      dl_add_rmsnorm_quant; the GEMM skips its activation
@@ -145,7 +148,9 @@ dl_status dl_fc13_swiglu(const uint16_t* x, int M, int K, const uint8_t* w_packe
  *     loads the library until the process exits.  M > 64 or M*K > 64*8192
  *     returns DL_ERR_WORKSPACE before anything is launched.
  *   - `status` is an optional device uint32 that the caller zeroes; device-
- *     side errors (bit 1 timeout) are OR-ed into it.  NULL: not reported.
+ *     side errors (bit 1 timeout) are OR-ed into it.  NULL turns device-side
+ *     error reporting off for the call (a wait that runs out still ends the
+ *     kernel; the output is then undefined and nothing says so).
  *   - nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
  *     library routine is called.
  *   - the first call on a device looks the array's device address up

@@ -492,7 +492,10 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   const uint32_t rv_o_l = smem_u32(rv_o), rv_ml_l = smem_u32(rv_ml);
   if constexpr (F8) {
     cluster_wait();  // every receive barrier of the cluster is initialised
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S * cnt * (16 + 8)));
+    // (test hook: 16 bytes more are expected than the peers send, so the
+    // owner's bounded receive wait below runs out)
+    if (threadIdx.x == 0)
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S * cnt * (16 + 8) + (a.debug ? 16 : 0)));
   }
   for (int it = threadIdx.x; it < I; it += kAttnThreads) {
     const int rho = it / (D / 4);
@@ -528,8 +531,11 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     }
   }
   // every state of my items has landed in my receive buffer
+  bool recv_ok = true;
   if constexpr (F8) {
-    if (!mbar_wait_cluster(recv_bar, 0, budget)) set_status(a.status, kStatusTimeout);
+    cluster_arrive();  // this CTA's pushes are issued (waited for before the CTA exits)
+    recv_ok = mbar_wait_cluster(recv_bar, 0, budget);
+    if (!recv_ok) set_status(a.status, kStatusTimeout);
   } else {
     cluster_sync();
   }
@@ -630,8 +636,16 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
       }
     }
   }
-  // No trailing cluster barrier: once a CTA has received all of its items, no
-  // other CTA touches its shared memory.
+  // bf16 cache: no trailing cluster barrier; once a CTA has passed the cluster
+  // barrier above, every peer's stores into its shared memory have landed.
+  // FP8 cache: a CTA leaves only once every CTA of the cluster has issued its
+  // pushes, so that no peer can still store into the shared memory of a CTA
+  // whose bounded receive wait ran out; the bytes issued before that barrier
+  // are then given one more bounded wait to land.
+  if constexpr (F8) {
+    cluster_wait();
+    if (!recv_ok) (void)mbar_wait_cluster(recv_bar, 0, budget);
+  }
 }
 
 // ---- host side ----------------------------------------------------------------------

@@ -10,8 +10,9 @@
 // One thread-block cluster per sequence.  CTA r of the cluster scans the r-th
 // slice of the vocabulary for all T positions of its sequence; every
 // (logit, index) pair becomes one 64-bit key (order-preserving float bits above,
-// inverted index below), so an unsigned max picks the largest logit and, on a
-// tie, the lowest index -- whatever order the threads arrive in.  The cluster
+// with -0 taken as +0, inverted index below), so an unsigned max picks the
+// largest logit and, on a tie, the lowest index -- whatever order the threads
+// arrive in.  The cluster
 // merges the per-CTA maxima through distributed shared memory, and CTA 0
 // decides the accepted prefix and writes the results.
 #include "dl_device.cuh"
@@ -39,7 +40,10 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// -0 and +0 are the same logit value: -0 is keyed as +0, so that a tie between
+// them, like any other tie, goes to the lower index.
 __device__ __forceinline__ unsigned long long sv_key(uint32_t bf16_bits, int index) {
+  if (bf16_bits == 0x8000u) bf16_bits = 0u;
   return (static_cast<unsigned long long>(ordered_bits(__uint_as_float(bf16_bits << 16))) << 32) |
          static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(index));
 }

@@ -78,9 +78,13 @@ extern "C" dl_status dl_fc13_swiglu_static_ws(const uint16_t* x, int M, int K, c
   }
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool pdl = (flags & DL_FLAG_PDL) != 0;
-  cudaError_t e = dl::launch_act_quant(x, M, K, dl::ws_xq(scratch), dl::ws_sx(scratch), s, pdl);
+  // As in dl_fc13_swiglu: small inputs are quantised inside the GEMM, larger
+  // ones by the quantise kernel first; both write x_q and s_x to the array.
+  const bool fused = static_cast<long long>(M) * K <= dl::kFusedQuantMaxElems;
+  cudaError_t e = fused ? cudaSuccess : dl::launch_act_quant(x, M, K, dl::ws_xq(scratch), dl::ws_sx(scratch), s, pdl);
   if (e == cudaSuccess) {
     dl::GemmLaunch g{};
+    g.x = fused ? x : nullptr;
     g.w = w_packed;
     g.w_expert_bytes = 0;
     g.w_scale = w_scale;

@@ -62,16 +62,20 @@ def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.linalg.norm((got - ref).ravel()) / (den if den > 0 else 1.0))
 
 
-def check_gemm(got_bits: np.ndarray, ref: np.ndarray, what: str = "") -> dict:
+def check_gemm(got_bits: np.ndarray, ref: np.ndarray, what: str = "", slack=None) -> dict:
     """bf16 GEMM outputs vs the float64 oracle: relative L2 <= 1e-2 over the
     call, and max-abs <= 3e-2 against the bf16-rounded reference, where an
     element whose bf16 spacing exceeds 3e-2 may sit one spacing away (a
-    rounding-boundary flip of a correct fp32 result)."""
+    rounding-boundary flip of a correct fp32 result).  `slack`, when given, is
+    a per-element allowance added to both rules (a derived bound for inputs
+    whose e4m3 codes may legitimately differ at rounding ties)."""
     got = bf16_to_f64(got_bits)
     rl2 = rel_l2(got, ref)
     rb = bf16_round_f64(ref)
     diff = np.abs(got - rb)
     ulp = bf16_ulp(rb)
+    if slack is not None:
+        diff = np.maximum(diff - slack, 0.0)
     bad = (diff > GEMM_MAX_ABS) & ~((ulp > GEMM_MAX_ABS) & (diff <= ulp * 1.0000001))
     stats = {"rel_l2": rl2, "max_abs_vs_bf16ref": float(diff.max(initial=0.0)),
              "raw_max_abs": float(np.abs(got - ref).max(initial=0.0)), "n_bad": int(bad.sum())}

@@ -75,7 +75,8 @@ def test_verify4_full(cluster):
 
 def test_batch16x4_full_size_sampled_sequences():
     """16 sequences with lengths drawn in [1024, 16384]; the GPU computes all of
-    them, the oracle checks four."""
+    them, the oracle checks the longest and the shortest drawn sequence, the
+    first and the last, and two more."""
     wl = dg.WORKLOADS["batch16x4"]
     g = dg.rng(wl.seed)
     sl = dg.seq_lens_for(wl, g)
@@ -83,7 +84,10 @@ def test_batch16x4_full_size_sampled_sequences():
     scale = 1.0 / math.sqrt(wl.d)
     got = run_attn(q.ravel(), wl.Hq * wl.d, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, k, v, sl, scale, wl.cluster)
     got = got.reshape(wl.B, wl.T, wl.Hq, wl.d)
-    for b in (0, 5, 10, 15):
+    picks = [int(np.argmax(sl)), int(np.argmin(sl)), 0, wl.B - 1, 5, 10]
+    picks = sorted(set(picks))
+    assert int(np.argmax(sl)) in picks and len(picks) >= 4
+    for b in picks:
         ref = oracle.decode_attn(q[b:b + 1].ravel(), wl.Hq * wl.d, 1, wl.T, wl.Hq, wl.Hkv, wl.d, k[b:b + 1],
                                  v[b:b + 1], sl[b:b + 1], scale)
         helpers.check_attn(got[b:b + 1], ref, f"batch16x4 seq {b} L={sl[b]}")

@@ -75,15 +75,87 @@ def test_reference_arm_two_ranks_under_torchrun():
     assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
 
 
-def test_oracle_baseline_on_two_host_cores():
-    """The all-cores CPU baseline: two spawned single-threaded oracle processes,
-    each timing whole layers of its own copy of the inputs."""
+def test_oracle_baseline_on_two_host_threads():
+    """The all-cores CPU baseline: one layer at a time, its output columns and
+    query heads spread over two host threads."""
     sys.path.insert(0, ROOT)
     import bench
     from latency_decode_b200 import datagen as dg
-    us, reps = bench.time_oracle_all_cores(dg.WORKLOADS["tiny"], 0.3, 2)
-    assert us > 0 and reps >= 2
+    wl = dg.WORKLOADS["tiny"]
+    us, reps, secs = bench.time_oracle_threads(wl, bench.oracle_layer_inputs(wl), 0.3, 2)
+    assert us > 0 and reps >= 1 and secs > 0
     assert 1 <= bench.host_cores() <= 16
+
+
+@pytest.mark.parametrize("name", ["tiny", "verify4_small"])
+def test_sliced_oracle_layer_equals_the_whole_oracle_layer(name):
+    """Spreading a layer's output columns and query heads over threads changes
+    nothing: every slice is the oracle's own function on part of the weights
+    (or one head), so the outputs are identical bit for bit."""
+    import dataclasses
+    from concurrent.futures import ThreadPoolExecutor
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    from latency_decode_b200 import datagen as dg
+    if name == "tiny":
+        wl = dg.WORKLOADS["tiny"]
+    else:  # several query tokens, causal, grouped heads, at a size the oracle runs in seconds
+        wl = dataclasses.replace(dg.WORKLOADS["verify4"], name=name, K=256, N2=1024, Hq=8, Hkv=2, d=64, L=300,
+                                 Lcap=320)
+    inp = bench.oracle_layer_inputs(wl)
+    whole = bench.oracle_layer(wl, inp)
+    with ThreadPoolExecutor(max_workers=3) as pool:
+        sliced = bench.oracle_layer_sliced(wl, inp, bench.sliced_oracle_inputs(wl, inp, fc13_cols=96), pool)
+    for a, b in zip(whole, sliced):
+        assert a.shape == b.shape and np.array_equal(a, b)
+
+
+def test_replay_plan_runs_exactly_n_steps_in_multi_step_graphs():
+    """The bench replays CUDA graphs of `period` chained steps and one graph of
+    the remainder: exactly n steps, and no single-step graphs unless n itself
+    is 1 or leaves a remainder of 1."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.replay_plan(20, 24) == [20]        # fewer steps than the period: one graph of all of them
+    assert bench.replay_plan(24, 24) == [24]
+    assert bench.replay_plan(2000, 24) == [24] * 83 + [8]
+    assert bench.replay_plan(48, 24) == [24, 24]
+    assert bench.replay_plan(1, 24) == [1]
+    assert bench.replay_plan(0, 24) == []
+    for n in range(1, 200):
+        for period in (1, 2, 3, 8, 24):
+            plan = bench.replay_plan(n, period)
+            assert sum(plan) == n and all(1 <= L <= period for L in plan)
+            assert all(L == period for L in plan[:-1])
+
+
+def test_graph_replayer_captures_each_length_once_and_replays_in_order():
+    """GraphReplayer against a stand-in capture: the graph of length L holds
+    fn(0..L-1) (each starts again at replica 0), one capture per distinct
+    length, and run(n) executes exactly n steps."""
+    sys.path.insert(0, ROOT)
+    import bench
+    log, captures = [], []
+
+    class FakeGraph:
+        def __init__(self, idxs):
+            self.idxs = list(idxs)
+
+        def replay(self):
+            log.extend(self.idxs)
+
+    def capture(fn, idxs):
+        captures.append(len(idxs))
+        return FakeGraph(idxs)
+
+    rp = bench.GraphReplayer(lambda i: None, 6, capture).prepare(20)
+    assert sorted(captures) == [2, 6]
+    rp.run(20)
+    assert log == list(range(6)) * 3 + [0, 1]
+    assert rp.lengths(20) == [6, 2]
+    rp.run(20)
+    assert sorted(captures) == [2, 6]  # nothing captured again
 
 
 def test_recorded_traffic_matches_the_current_source_only(tmp_path, monkeypatch):

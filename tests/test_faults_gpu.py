@@ -90,6 +90,32 @@ def test_attention_timeout_is_reported_and_context_stays_usable():
     helpers.check_attn(host_u16(out), ref, "after timeout")
 
 
+def test_fp8kv_attention_timeouts_are_reported_and_context_stays_usable():
+    """FP8-cache attention under the test hook: the producer withholds its last
+    tile, and each owner CTA expects 16 bytes more than its peers push, so both
+    the tile wait and the merge's receive wait run out.  Every CTA still waits
+    at the cluster barrier for its peers' pushes before it exits; the status is
+    reported and the next normal call matches the oracle."""
+    g = np.random.default_rng(5)
+    B, T, Hq, Hkv, d, L = 1, 4, 8, 2, 128, 320
+    q = dg.bf16_normal(g, (B, T, Hq, d))
+    kc = g.integers(0, 0x7E, size=(B, Hkv, L, d)).astype(np.uint8)
+    vt = g.integers(0, 0x7E, size=(B, Hkv, d, L)).astype(np.uint8)
+    sl = np.int32([L])
+    s_k, s_v = np.float32(0.01), np.float32(0.02)
+    out = torch.empty((B, T, Hq, d), dtype=torch.int16, device="cuda")
+    n = dl.dl_decode_attn_fp8kv_workspace_bytes(B, T, Hq, Hkv, d, L, 4)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    args = (dev_u16(q), Hq * d, B, T, Hq, Hkv, d, dev_u8(kc), dev_u8(vt), dev_f32([s_k, s_v]), L, dev_i32(sl),
+            1 / math.sqrt(d), 4, out, ws, n)
+    assert dl.dl_decode_attn_fp8kv(*args, flags=dl.DL_FLAG_PDL | dl.DL_FLAG_DEBUG_TIMEOUT) == dl.DL_OK
+    assert dl.dl_read_status(ws) == dl.DL_ERR_TIMEOUT
+    dl.check(dl.dl_decode_attn_fp8kv(*args))
+    assert dl.dl_read_status(ws) == dl.DL_OK
+    ref = oracle.decode_attn_fp8kv(q.ravel(), Hq * d, B, T, Hq, Hkv, d, kc, vt, sl, 1 / math.sqrt(d), s_k, s_v)
+    helpers.check_attn(host_u16(out), ref, "after timeout")
+
+
 def test_moe_timeout_is_reported():
     g = np.random.default_rng(6)
     T, E, K, N2 = 4, 3, 512, 256

@@ -20,6 +20,7 @@ from helpers import dev_f32, dev_i32, dev_u8, dev_u16, host_u16, new_ws
 from latency_decode_b200 import build as dl_build
 from latency_decode_b200 import datagen as dg
 from latency_decode_b200 import dl
+from layer_chain_ref import chain_tolerance, oracle_full_layer
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not helpers.gpu_available(), reason="needs a CUDA GPU")]
@@ -236,6 +237,48 @@ def test_add_rmsnorm_quant_zero_rows_and_large_eps():
     assert sx0 == 1.0 and not xq0.any()  # all-zero input: s_x = 1, codes 0
 
 
+def tie_flip_bound(y_ref, xq_ref, sx, w, s_w, swiglu):
+    """Largest change of each output that the producer's admissible code flips
+    can cause, from the oracle's own quantities only.
+
+    The producer's codes may differ from the oracle's only where the oracle's
+    fp32 product y*inv sits at a rounding midpoint of two e4m3 values (to 1e-5
+    relative, as codes_close checks).  A flip there moves the code by one e4m3
+    spacing, delta = 2|p - dec(c)|.  For one token row m and output column n
+    the pre-activation then moves by at most
+        D[m, n] = s_x * s_w * sum over tie positions k of delta[m, k] * |dec(W[n, k])|.
+    A plain output moves by D.  For SwiGLU, out = silu(g) u with |silu'| <= 1.1,
+    so over the box g +- Dg, u +- Du it moves by at most
+        1.1 Dg (|u| + Du) + (|silu(g)| + 1.1 Dg) Du.
+    Returns that bound, shaped like the output ([M, N] or [M, F])."""
+    yf = y_ref.astype(np.float32)
+    amax = np.float32(np.abs(yf).max())
+    inv = np.float32(448.0) / amax
+    p = (yf * inv).astype(np.float64)
+    table = e4m3_values(np.arange(256, dtype=np.uint8))
+    finite = np.isfinite(table)
+    grid = np.unique(table[finite])
+    v = e4m3_values(xq_ref)
+    # the neighbouring e4m3 value on the side of p, and the midpoint towards it
+    idx = np.searchsorted(grid, v)
+    up = grid[np.minimum(idx + 1, grid.size - 1)]
+    dn = grid[np.maximum(idx - 1, 0)]
+    nb = np.where(p >= v, up, dn)
+    mid = (v + nb) / 2
+    tie = np.abs(p - mid) <= 1e-5 * np.maximum(np.abs(mid), 1e-30)
+    delta = np.where(tie, np.abs(nb - v), 0.0)
+    wv = np.abs(e4m3_values(w))
+    D = float(sx) * float(s_w) * (delta @ wv.T)
+    if not swiglu:
+        return D
+    F = w.shape[0] // 2
+    y = float(sx) * float(s_w) * (e4m3_values(xq_ref) @ e4m3_values(w).T)
+    g, u = y[:, :F], y[:, F:]
+    Dg, Du = D[:, :F], D[:, F:]
+    silu = g / (1.0 + np.exp(-g))
+    return 1.1 * Dg * (np.abs(u) + Du) + (np.abs(silu) + 1.1 * Dg) * Du
+
+
 EPS_EXACT = 2.0 ** -40  # below half an fp32 ulp of mean(h^2) >= 1/4: rsqrt sees mean(h^2) alone
 
 
@@ -255,9 +298,10 @@ def test_norm_then_gemm_through_the_workspace(name, inputs):
     with DL_FLAG_XQ_READY (x = NULL), chained under PDL on one stream; the
     oracle checks 128 sampled output columns of every token.  'exact' inputs
     make the two sides' codes identical, so the GEMM output is held to the
-    element-wise GEMM rule; with 'random' inputs a code at a rounding tie may
-    differ (see codes_close), which moves an output by up to a few bf16 steps,
-    so only the relative L2 bound applies there."""
+    element-wise GEMM rule.  With 'random' inputs a code at a rounding tie may
+    differ (codes_close checks that every difference is such a tie); the GEMM
+    rule then holds with each output's allowance widened by tie_flip_bound,
+    the most that the admissible flips can move it."""
     wl = dg.WORKLOADS[name]
     g = dg.rng(500 + wl.seed)
     if inputs == "exact":
@@ -285,11 +329,15 @@ def test_norm_then_gemm_through_the_workspace(name, inputs):
     sub = np.ascontiguousarray(np.concatenate([w13[cols], w13[F + cols]]))
     ref = oracle.fc13_swiglu_q(xq_ref, sx_ref, sub, s13)
     got = host_u16(out)[:, cols]
+    xq_gpu = ws[256:256 + wl.M * wl.K].cpu().numpy().reshape(wl.M, wl.K)
     if inputs == "exact":
-        assert np.array_equal(ws[256:256 + wl.M * wl.K].cpu().numpy().reshape(wl.M, wl.K), xq_ref)
+        assert np.array_equal(xq_gpu, xq_ref)
         helpers.check_gemm(got, ref, f"{name} norm -> fc13 (exact rows)")
     else:
-        assert helpers.rel_l2(helpers.bf16_to_f64(got), ref) <= helpers.GEMM_REL_L2
+        _, y_ref, _, _ = oracle.add_rmsnorm_quant(x, r, gam, eps)
+        codes_close(xq_gpu, xq_ref, y_ref, f"{name} norm codes")
+        slack = tie_flip_bound(y_ref, xq_ref, sx_ref, sub, s13, swiglu=True)
+        helpers.check_gemm(got, ref, f"{name} norm -> fc13 (random rows)", slack=slack)
 
 
 def test_xq_ready_plain_and_qkv_entries_read_the_producer_output():
@@ -314,29 +362,8 @@ def test_xq_ready_plain_and_qkv_entries_read_the_producer_output():
 
 # ------------------------------------------------------------ whole layer --
 
-def oracle_full_layer(inp, wl, eps):
-    """The layer restated with oracle steps only; every hand-over between steps
-    is rounded to bf16 (the storage format between kernels)."""
-    rnd = lambda a: oracle.f64_to_bf16(a)
-    h1, _, xq1, sx1 = oracle.add_rmsnorm_quant(inp["x"], inp["h"], inp["g1"], eps)
-    qkv = rnd(oracle.fc_qkv_scale_q(xq1, sx1, inp["w_qkv"], inp["s_qkv"], wl.Hq, wl.Hkv, wl.d, inp["q_scale"]))
-    att = rnd(oracle.decode_attn(qkv.ravel(), wl.n_qkv, wl.B, wl.T, wl.Hq, wl.Hkv, wl.d, inp["k_cache"],
-                                 inp["v_cache"], inp["seq_lens"], 1.0)).reshape(wl.M, wl.k_o)
-    a = rnd(oracle.linear(att, inp["w_o"], inp["s_o"]))
-    h2, _, xq2, sx2 = oracle.add_rmsnorm_quant(a, h1, inp["g2"], eps)
-    f = rnd(oracle.fc13_swiglu_q(xq2, sx2, inp["w13"], inp["s13"]))
-    return oracle.linear(f, inp["w2"], inp["s2"]), h2
-
-
-@pytest.mark.parametrize("name", ["tiny", "layer_b1"])
-def test_full_layer_chain(name):
-    """The seven-kernel layer under PDL against the oracle chain.  Intermediate
-    bf16 and e4m3 roundings can differ at a few elements (each side rounds its
-    own intermediate), so the layer output is held to relative L2 <= 2e-2 and
-    the residual stream, which passes through one GEMM less, to 1e-2."""
+def run_full_layer(wl, inp):
     from latency_decode_b200.layer import FullDecodeLayer
-    wl = dg.WORKLOADS[name]
-    inp = dg.full_layer_inputs(wl)
     lay = FullDecodeLayer(dev_u8(inp["w_qkv"]), inp["s_qkv"], dev_u8(inp["w_o"]), inp["s_o"], dev_u8(inp["w13"]),
                           inp["s13"], dev_u8(inp["w2"]), inp["s2"], dev_u16(inp["g1"]), dev_u16(inp["g2"]),
                           Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, q_scale=inp["q_scale"], M=wl.M, B=wl.B, T=wl.T,
@@ -344,11 +371,40 @@ def test_full_layer_chain(name):
     h = dev_u16(inp["h"])
     lay.step(dev_u16(inp["x"]), h, dev_u16(inp["k_cache"]), dev_u16(inp["v_cache"]), dev_i32(inp["seq_lens"]))
     lay.read_status()
+    return helpers.bf16_to_f64(host_u16(lay.y)), host_u16(h)
+
+
+@pytest.mark.parametrize("name", ["tiny", "layer_b1"])
+def test_full_layer_chain(name):
+    """The seven-kernel layer under PDL against the oracle chain.  Each later
+    stage re-quantises to e4m3, so an attention output that is right within its
+    tolerance still moves downstream codes; the bound is the oracle chain's own
+    spread under attention noise at the attention tolerance
+    (layer_chain_ref.chain_tolerance)."""
+    wl = dg.WORKLOADS[name]
+    inp = dg.full_layer_inputs(wl)
+    y, h = run_full_layer(wl, inp)
     y_ref, h_ref = oracle_full_layer(inp, wl, 1e-5)
-    y = helpers.bf16_to_f64(host_u16(lay.y))
+    tol_y, tol_h = chain_tolerance(inp, wl, 1e-5, y_ref, h_ref)
     assert np.isfinite(y).all()
-    assert helpers.rel_l2(y, y_ref) <= 2e-2, helpers.rel_l2(y, y_ref)
-    assert helpers.rel_l2(helpers.bf16_to_f64(host_u16(h)), helpers.bf16_to_f64(h_ref)) <= 1e-2
+    assert helpers.rel_l2(y, y_ref) <= tol_y, (helpers.rel_l2(y, y_ref), tol_y)
+    assert helpers.rel_l2(helpers.bf16_to_f64(h), helpers.bf16_to_f64(h_ref)) <= tol_h
+
+
+@pytest.mark.parametrize("name", ["tiny", "layer_b1"])
+def test_full_layer_chain_identical_keys_at_the_gemm_bound(name):
+    """With every cached key equal, the attention output is the mean of the
+    visible values, which both sides compute to within a bf16 rounding; the
+    seven-kernel chain then holds the GEMM bound (relative L2 <= 1e-2) at its
+    output and on the residual stream."""
+    wl = dg.WORKLOADS[name]
+    inp = dg.full_layer_inputs(wl)
+    inp["k_cache"] = np.ascontiguousarray(np.broadcast_to(inp["k_cache"][:, :, :1, :], inp["k_cache"].shape))
+    y, h = run_full_layer(wl, inp)
+    y_ref, h_ref = oracle_full_layer(inp, wl, 1e-5)
+    assert np.isfinite(y).all()
+    assert helpers.rel_l2(y, y_ref) <= helpers.GEMM_REL_L2, helpers.rel_l2(y, y_ref)
+    assert helpers.rel_l2(helpers.bf16_to_f64(h), helpers.bf16_to_f64(h_ref)) <= helpers.GEMM_REL_L2
 
 
 # ------------------------------------- RMSNorm producer + GEMM in one call --
@@ -357,8 +413,9 @@ def test_full_layer_chain(name):
 @pytest.mark.parametrize("inputs", ["exact", "random"])
 def test_rmsnorm_fused_into_fc13(M, inputs):
     """dl_rmsnorm_fc13_swiglu (producer kernel + GEMM in one call).  Exact rows:
-    codes identical to the oracle's, element-wise GEMM rule; random rows:
-    relative L2 (a code at a rounding tie may differ)."""
+    codes identical to the oracle's, element-wise GEMM rule; random rows: codes
+    may differ only at rounding ties, and the GEMM rule holds with the
+    allowance widened by tie_flip_bound."""
     K, N2 = 2048, 512
     g = np.random.default_rng(700 + M + (inputs == "exact") * 50)
     if inputs == "exact":
@@ -383,11 +440,15 @@ def test_rmsnorm_fused_into_fc13(M, inputs):
     h_ref, _, xq_ref, sx_ref = oracle.add_rmsnorm_quant(x, r, gam, eps)
     assert np.array_equal(host_u16(hd), h_ref)
     ref = oracle.fc13_swiglu_q(xq_ref, sx_ref, w, s_w)
+    xq_gpu = ws[256:256 + M * K].cpu().numpy().reshape(M, K)
     if inputs == "exact":
-        assert np.array_equal(ws[256:256 + M * K].cpu().numpy().reshape(M, K), xq_ref)
+        assert np.array_equal(xq_gpu, xq_ref)
         helpers.check_gemm(host_u16(out), ref, f"fused norm fc13 M={M}")
     else:
-        assert helpers.rel_l2(helpers.bf16_to_f64(host_u16(out)), ref) <= helpers.GEMM_REL_L2
+        _, y_ref, _, _ = oracle.add_rmsnorm_quant(x, r, gam, eps)
+        codes_close(xq_gpu, xq_ref, y_ref, f"fused norm codes M={M}")
+        slack = tie_flip_bound(y_ref, xq_ref, sx_ref, w, s_w, swiglu=True)
+        helpers.check_gemm(host_u16(out), ref, f"fused norm fc13 M={M} (random rows)", slack=slack)
 
 
 @pytest.mark.parametrize("M", [1, 5])

@@ -547,6 +547,29 @@ def test_spec_verify_hand_example(golden_dir):
     assert em[0].tolist() == gold["emitted"]
 
 
+def _signed_zero_logits(gold):
+    """Logits of the signed-zero fixture as bf16 bits: -1.0 everywhere, then
+    the listed -0 (0x8000) and +0 (0x0000) entries."""
+    T, V = len(gold["target_ids"]), gold["V"]
+    lg = np.full((1, T, V), dg.bf16_bits(np.float32([-1.0]))[0], dtype=np.uint16)
+    for t, v in gold["neg_zero"]:
+        lg[0, t, v] = 0x8000
+    for t, v in gold["pos_zero"]:
+        lg[0, t, v] = 0x0000
+    return lg
+
+
+def test_spec_verify_signed_zero_tie(golden_dir):
+    """-0 and +0 are one value: the lower index wins, whatever its sign (numpy's
+    argmax on the decoded values agrees)."""
+    gold = json.load(open(os.path.join(golden_dir, "spec_verify_signed_zero.json")))
+    lg = _signed_zero_logits(gold)
+    tid, nacc, em = oracle.spec_verify_greedy(lg, np.array([gold["draft"]], dtype=np.int32))
+    assert tid[0].tolist() == gold["target_ids"]
+    assert tid[0].tolist() == np.argmax(_bf16_torch(lg)[0], axis=1).tolist()
+    assert int(nacc[0]) == gold["n_accepted"] and em[0].tolist() == gold["emitted"]
+
+
 def test_spec_verify_matches_numpy_argmax_and_brute_force_acceptance():
     g = np.random.default_rng(71)
     B, T, V = 6, 4, 1000

@@ -77,6 +77,29 @@ def test_pages_worked_example(golden_dir):
     assert em[0].tolist() == gold["emitted"] and int(sl[0]) == 1000 - 1
 
 
+def test_signed_zero_tie_lowest_index_wins(golden_dir):
+    """The largest logit is 0, present as -0 before +0 (and +0 before -0): the
+    lower index wins, as in the oracle; also with the zeros in different CTA
+    slices of the full vocabulary."""
+    gold = json.load(open(os.path.join(golden_dir, "spec_verify_signed_zero.json")))
+    T, V = len(gold["target_ids"]), gold["V"]
+    lg = np.full((1, T, V), dg.bf16_bits(np.float32([-1.0]))[0], dtype=np.uint16)
+    for t, v in gold["neg_zero"]:
+        lg[0, t, v] = 0x8000
+    for t, v in gold["pos_zero"]:
+        lg[0, t, v] = 0x0000
+    tid, nacc, em, _ = run_verify(lg, np.array([gold["draft"]], np.int32))
+    assert tid[0].tolist() == gold["target_ids"] and int(nacc[0]) == gold["n_accepted"]
+    assert em[0].tolist() == gold["emitted"]
+    big = np.full((2, 3, dg.VOCAB), dg.bf16_bits(np.float32([-2.0]))[0], dtype=np.uint16)
+    big[0, 0, 7], big[0, 0, 150001] = 0x8000, 0x0000        # -0 first, far apart
+    big[0, 1, 100], big[0, 1, 190000] = 0x0000, 0x8000      # +0 first
+    big[0, 2, 24], big[0, 2, 25] = 0x8000, 0x0000           # inside one 16-byte vector
+    big[1, :, 202047] = 0x0000
+    big[1, :, 202046] = 0x8000
+    check(big, np.array([[7, 100], [202046, 5]], np.int32), None, "signed zeros")
+
+
 @pytest.mark.parametrize("B,T,V", [(1, 4, 1000), (3, 4, 4096), (16, 4, 32000), (64, 2, 2048), (5, 8, 800),
                                    (2, 32, 128), (1, 1, 64)])
 def test_every_accept_length(B, T, V):
