@@ -48,6 +48,7 @@ namespace dl {
 // softmax latency) for clusters of up to 8 CTAs; W = 4 (two CTAs per SM where
 // they fit) for 16-CTA clusters, which pack onto the GPCs only that way.
 constexpr int kAttnMaxSplits = 16;    // clusters per (b, kv head)
+constexpr int kAttnMaxCluster = 16;   // CTAs per cluster
 constexpr int kLazyRescale = 8;       // log2 headroom before the running max is raised
 
 struct AttnArgs {
@@ -500,24 +501,30 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
   for (int it = threadIdx.x; it < I; it += kAttnThreads) {
     const int rho = it / (D / 4);
     const int c4 = it - rho * (D / 4);
+    // Every load is issued up front and unconditionally (all are in bounds), so
+    // the W states cost one shared-memory round trip rather than one per warp;
+    // a warp without visible keys (l = 0) gets weight 0.
+    float mw[kAttnConsumers], lw[kAttnConsumers];
+    float4 ow[kAttnConsumers];
+#pragma unroll
+    for (int w = 0; w < kAttnConsumers; ++w) {
+      mw[w] = wm[w * R + rho];
+      lw[w] = wl[w * R + rho];
+      ow[w] = *reinterpret_cast<const float4*>(wo + (w * R + rho) * DP + c4 * 4);
+    }
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kAttnConsumers; ++w)
-      if (wl[w * R + rho] > 0.0f) M = fmaxf(M, wm[w * R + rho]);
+    for (int w = 0; w < kAttnConsumers; ++w) M = lw[w] > 0.0f ? fmaxf(M, mw[w]) : M;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.0f;
 #pragma unroll
     for (int w = 0; w < kAttnConsumers; ++w) {
-      const float lw = wl[w * R + rho];
-      if (lw > 0.0f) {
-        const float f = ex2(wm[w * R + rho] - M);
-        const float4 v = *reinterpret_cast<const float4*>(wo + (w * R + rho) * DP + c4 * 4);
-        acc.x += v.x * f;
-        acc.y += v.y * f;
-        acc.z += v.z * f;
-        acc.w += v.w * f;
-        lsum += lw * f;
-      }
+      const float f = lw[w] > 0.0f ? ex2(mw[w] - M) : 0.0f;
+      acc.x += ow[w].x * f;
+      acc.y += ow[w].y * f;
+      acc.z += ow[w].z * f;
+      acc.w += ow[w].w * f;
+      lsum += lw[w] * f;
     }
     const int owner = it / Q;
     const uint32_t slot_i = static_cast<uint32_t>(rank * Q + (it - owner * Q));
@@ -548,21 +555,35 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     const int it = my0 + k;
     const int rho = it / (D / 4);
     const int c4 = it - rho * (D / 4);
+    // All (m, l) first, then the o states in groups of 4, each group's loads
+    // issued together; indices past S are clamped to S - 1 (in bounds) and get
+    // weight 0, so no load sits behind a branch.
+    float mp[kAttnMaxCluster], lp[kAttnMaxCluster];
+#pragma unroll
+    for (int p = 0; p < kAttnMaxCluster; ++p) {
+      const float2 ml = rv_ml[(p < S ? p : S - 1) * Q + k];
+      mp[p] = ml.x;
+      lp[p] = p < S ? ml.y : 0.0f;
+    }
     float M = -INFINITY;
-    for (int p = 0; p < S; ++p)
-      if (rv_ml[p * Q + k].y > 0.0f) M = fmaxf(M, rv_ml[p * Q + k].x);
+#pragma unroll
+    for (int p = 0; p < kAttnMaxCluster; ++p) M = lp[p] > 0.0f ? fmaxf(M, mp[p]) : M;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.0f;
-    for (int p = 0; p < S; ++p) {
-      const float lp = rv_ml[p * Q + k].y;
-      if (lp > 0.0f) {
-        const float f = ex2(rv_ml[p * Q + k].x - M);
-        const float4 v = rv_o[p * Q + k];
-        acc.x += v.x * f;
-        acc.y += v.y * f;
-        acc.z += v.z * f;
-        acc.w += v.w * f;
-        lsum += lp * f;
+#pragma unroll
+    for (int p0 = 0; p0 < kAttnMaxCluster; p0 += 4) {
+      if (p0 >= S) break;
+      float4 v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = rv_o[(p0 + q < S ? p0 + q : S - 1) * Q + k];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float f = lp[p0 + q] > 0.0f ? ex2(mp[p0 + q] - M) : 0.0f;
+        acc.x += v[q].x * f;
+        acc.y += v[q].y * f;
+        acc.z += v[q].z * f;
+        acc.w += v[q].w * f;
+        lsum += lp[p0 + q] * f;
       }
     }
     if (a.P == 1) {
@@ -605,24 +626,37 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         const int it = my0 + k;
         const int rho = it / (D / 4);
         const int c4 = it - rho * (D / 4);
-        float M = -INFINITY;
-        for (int p = 0; p < a.P; ++p) {
-          const float* ml = a.part_ml + (((head * a.P + p) * S + rank) * R + rho) * 2;
-          if (__ldcg(ml + 1) > 0.0f) M = fmaxf(M, __ldcg(ml));
+        // as in the owner merge: every load of a group issued together, indices
+        // past P clamped and weighted 0
+        float mq[kAttnMaxSplits], lq[kAttnMaxSplits];
+#pragma unroll
+        for (int p = 0; p < kAttnMaxSplits; ++p) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+              a.part_ml + (((head * a.P + (p < a.P ? p : a.P - 1)) * S + rank) * R + rho) * 2));
+          mq[p] = ml.x;
+          lq[p] = p < a.P ? ml.y : 0.0f;
         }
+        float M = -INFINITY;
+#pragma unroll
+        for (int p = 0; p < kAttnMaxSplits; ++p) M = lq[p] > 0.0f ? fmaxf(M, mq[p]) : M;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float lsum = 0.0f;
-        for (int p = 0; p < a.P; ++p) {
-          const float* ml = a.part_ml + (((head * a.P + p) * S + rank) * R + rho) * 2;
-          const float lq = __ldcg(ml + 1);
-          if (lq > 0.0f) {
-            const float f = ex2(__ldcg(ml) - M);
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((head * a.P + p) * I + it) * 4));
-            acc.x += v.x * f;
-            acc.y += v.y * f;
-            acc.z += v.z * f;
-            acc.w += v.w * f;
-            lsum += lq * f;
+#pragma unroll
+        for (int p0 = 0; p0 < kAttnMaxSplits; p0 += 4) {
+          if (p0 >= a.P) break;
+          float4 v[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            v[q] = __ldcg(reinterpret_cast<const float4*>(
+                a.part_o + ((head * a.P + (p0 + q < a.P ? p0 + q : a.P - 1)) * I + it) * 4));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float f = lq[p0 + q] > 0.0f ? ex2(mq[p0 + q] - M) : 0.0f;
+            acc.x += v[q].x * f;
+            acc.y += v[q].y * f;
+            acc.z += v[q].z * f;
+            acc.w += v[q].w * f;
+            lsum += lq[p0 + q] * f;
           }
         }
         const float inv = lsum > 0.0f ? out_scale / lsum : 0.0f;
