@@ -257,14 +257,21 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
     if (threadIdx.x == 0) pdl_trigger();
 
     // Q^T fragments (B operand of S^T = K Q^T), column n = query row g of tile nt,
-    // staged once in shared memory by the four consumer warps.
-    for (int f = threadIdx.x; f < KS * NT * 32; f += 32 * kAttnConsumers) {
+    // staged once in shared memory by the consumer warps.  Each thread's QI
+    // entries are loaded in one unrolled pass before any is stored, so the
+    // staging costs one memory round trip, not one per entry.
+    constexpr int QN = KS * NT * 32;                       // entries
+    constexpr int QI = (QN + 32 * kAttnConsumers - 1) / (32 * kAttnConsumers);
+    uint2 qv[QI];
+#pragma unroll
+    for (int i = 0; i < QI; ++i) {
+      const int f = threadIdx.x + i * 32 * kAttnConsumers;
       const int ln = f & 31;
       const int nt = (f >> 5) % NT;
       const int ks = (f >> 5) / NT;
       const int rho = nt * 8 + (ln >> 2);
-      uint2 v = make_uint2(0u, 0u);
-      if (rho < a.R) {
+      qv[i] = make_uint2(0u, 0u);
+      if (f < QN && rho < a.R) {
         const int t = rho / a.G;
         const int hq = hk * a.G + rho % a.G;
         const uint16_t* qrow =
@@ -272,14 +279,18 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         if (F8) {  // k-step ks, thread t: physical d = 32t + 4ks + e; bf16 -> f16
           const int d0 = 32 * (ln & 3) + 4 * ks;
           const uint32_t w0 = ld_b32(qrow + d0), w1 = ld_b32(qrow + d0 + 2);
-          v.x = pack_f16x2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
-          v.y = pack_f16x2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
+          qv[i].x = pack_f16x2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
+          qv[i].y = pack_f16x2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
         } else {
-          v.x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
-          v.y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
+          qv[i].x = ld_b32(qrow + ks * 16 + 2 * (ln & 3));
+          qv[i].y = ld_b32(qrow + ks * 16 + 8 + 2 * (ln & 3));
         }
       }
-      qs[f] = v;
+    }
+#pragma unroll
+    for (int i = 0; i < QI; ++i) {
+      const int f = threadIdx.x + i * 32 * kAttnConsumers;
+      if (f < QN) qs[f] = qv[i];
     }
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kAttnConsumers) : "memory");
 

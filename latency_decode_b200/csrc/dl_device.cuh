@@ -198,6 +198,11 @@ __device__ __forceinline__ void dsmem_st_async_f32x4(uint32_t addr, float4 v, ui
                "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
                : "memory");
 }
+__device__ __forceinline__ void dsmem_st_async_f32(uint32_t addr, float x, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
+               "r"(__float_as_uint(x)), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void dsmem_st_async_f32x2(uint32_t addr, float x, float y, uint32_t bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
                "f"(x), "f"(y), "r"(bar)

@@ -60,6 +60,7 @@ struct GemmArgs {
   int bsm_bytes;
   int tmem_cols;
   int recv_bytes;             // > 0: split-K partials are pushed into a dedicated receive buffer
+  int coop;                   // fused quantiser: the cluster shares the amax (each CTA reads its K slice)
   int debug;
 };
 
@@ -68,6 +69,7 @@ struct GemmMisc {
   int abort;
   float sx;                   // activation scale used by the epilogue
   float wmax[2];              // per-warp |x| maxima of the fused quantiser
+  float peer_amax[8];         // cooperative quantiser: the slice maxima of the cluster's CTAs
   int n_tok;
   int expert;
   int tokens[kMaxTok];
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   uint8_t* ring = smem;
   uint8_t* bsm = ring + a.stages * kSubBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(bsm + a.bsm_bytes);
-  GemmMisc* misc = reinterpret_cast<GemmMisc*>(bars + 2 * a.stages + 2 + 2 * kBStages);
+  GemmMisc* misc = reinterpret_cast<GemmMisc*>(bars + 2 * a.stages + 3 + 2 * kBStages);
   float* recv = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(misc) + ((sizeof(GemmMisc) + 15) & ~15));
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8u * a.stages;
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   const uint32_t done = xready + 8u;
   const uint32_t bfull0 = done + 8u;                 // B ring (streamed activations)
   const uint32_t bempty0 = bfull0 + 8u * kBStages;
+  const uint32_t amaxbar = bempty0 + 8u * kBStages;  // cooperative quantiser: the cluster's slice maxima
   // Fused quantiser: the whole B slice is written once (xready).  Otherwise the
   // e4m3 activations stream through a kBStages ring beside the weight ring.
   const bool stream_b = a.x == nullptr;
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       mbar_init(bfull0 + 8u * s, 64);
       mbar_init(bempty0 + 8u * s, 1);
     }
+    mbar_init(amaxbar, 1);
     misc->abort = 0;
     fence_mbar_init();
   }
@@ -224,6 +228,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
+  // Cooperative quantiser: first phase of a split cluster barrier.  Every
+  // thread arrives here; the stagers wait before they store into a peer's
+  // shared memory (so every peer's barriers are initialised), the other warps
+  // wait before the epilogue's cluster barrier.
+  if (a.coop) cluster_arrive();
 
   if (warp == 0) {
     // ---- weight producer ----
@@ -314,6 +323,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     // them by 64 chunks without a division
     const int row_t = t / per_row;
     const int rem_t = t - row_t * per_row;
+    if (a.x != nullptr) {
+      // The B operand's token-padding rows (n_tok .. npad-1) stay zero: write the
+      // whole slice as zeros now, before the wait, so that after it only the
+      // real rows are quantised.
+      for (int c = t; c < chunks; c += 64) *reinterpret_cast<uint4*>(bsm + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
     pdl_wait();  // x (or x_q and s_x) is written by the preceding kernel
     pdl_trigger();
     if (a.x != nullptr) {
@@ -326,8 +341,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       const int nv = (a.M * a.K) >> 3;
       // This thread's first kKeep chunks of the CTA's K slice are loaded into
       // registers in the same batch as the amax loads, so quantising them
-      // needs no second trip to memory.
-      constexpr int kKeep = 4;
+      // needs no second trip to memory.  With the cooperative quantiser these
+      // chunks are the whole slice, and the only loads.
+      constexpr int kKeep = 5;
       uint4 keep[2 * kKeep];
       {
         int row = row_t, rem = rem_t;
@@ -350,10 +366,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
         }
       }
       // amax over all of x: 16 independent 16-byte loads in flight per thread per
-      // round, so x (10 KB at batch 1) arrives in one memory round trip.
+      // round, so x (10 KB at batch 1) arrives in one memory round trip.  The
+      // cooperative quantiser takes the amax of its slice (the kept chunks)
+      // and exchanges it with the cluster instead.
       constexpr int kBatch = 16;
       float m = 0.0f;
-      for (int base = t; base < nv; base += 64 * kBatch) {
+      if (a.coop) {
+#pragma unroll
+        for (int j = 0; j < 2 * kKeep; ++j) m = fmaxf(m, absmax8(keep[j]));
+      }
+      for (int base = a.coop ? nv : t; base < nv; base += 64 * kBatch) {
         uint4 u[kBatch];
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
@@ -367,37 +389,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (lane == 0) misc->wmax[warp - 2] = m;
       asm volatile("bar.sync 1, 64;" ::: "memory");  // the two stager warps only
-      const float amax = fmaxf(misc->wmax[0], misc->wmax[1]);
+      float amax = fmaxf(misc->wmax[0], misc->wmax[1]);
+      if (a.coop) {
+        // The S slices of the cluster cover all of x: each CTA sends its slice
+        // maximum to every CTA of the cluster (itself included), counted on the
+        // receiver's amaxbar, and takes the maximum of the S values it receives.
+        cluster_wait();  // every CTA of the cluster has initialised its barriers
+        if (t == 0) {
+          mbar_arrive_expect_tx(amaxbar, static_cast<uint32_t>(4 * S));
+          const uint32_t slot = smem_u32(&misc->peer_amax[rank]);
+          for (int p = 0; p < S; ++p)
+            dsmem_st_async_f32(dsmem_addr(slot, static_cast<uint32_t>(p)), amax,
+                               dsmem_addr(amaxbar, static_cast<uint32_t>(p)));
+        }
+        if (!mbar_wait_cluster(amaxbar, 0, budget)) {
+          set_status(a.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+        amax = 0.0f;
+        for (int p = 0; p < S; ++p) amax = fmaxf(amax, misc->peer_amax[p]);
+      }
       const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 0.0f;
       if (t == 0) misc->sx = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
       const bool publish = blockIdx.y == 0 && blockIdx.z == 0;  // one CTA column writes x_q / s_x
       if (publish && rank == 0 && t == 0) *a.s_x = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      for (int c = t, j = 0, row = row_t, rem = rem_t; c < chunks; c += 64, ++j) {
+      // This thread's chunks, in order; rows only grow with c, so the work ends
+      // at the first padding row.  The first kKeep chunks come from registers,
+      // in one unrolled block (independent chains), the rest are loaded here.
+      auto put = [&](int row, int rem, uint4 v) {
         const int kbl = rem >> 3;
         const int ch = rem & 7;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < n_tok && amax > 0.0f) {
-          uint4 u0, u1;
-          if (j < kKeep) {
-#pragma unroll
-            for (int q = 0; q < kKeep; ++q)
-              if (q == j) {
-                u0 = keep[2 * q];
-                u1 = keep[2 * q + 1];
-              }
-          } else {
-            const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + kbl) * 128 + ch * 16) >> 3);
-            u0 = __ldcg(src);
-            u1 = __ldcg(src + 1);
-          }
-          v = make_uint4(quant4(u0.x, u0.y, inv), quant4(u0.z, u0.w, inv), quant4(u1.x, u1.y, inv),
-                         quant4(u1.z, u1.w, inv));
-        }
-        if (publish && row < n_tok)
+        if (publish)
           *reinterpret_cast<uint4*>(const_cast<uint8_t*>(a.xq) + static_cast<long long>(row) * a.K +
                                     (kb0 + kbl) * 128 + ch * 16) = v;
-        uint8_t* dst = bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((ch ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = v;
+        *reinterpret_cast<uint4*>(bsm + kbl * npad * 128 + (row >> 3) * 1024 + (row & 7) * 128 +
+                                  ((ch ^ (row & 7)) << 4)) = v;
+      };
+      auto quant16 = [&](uint4 u0, uint4 u1) {
+        return amax > 0.0f ? make_uint4(quant4(u0.x, u0.y, inv), quant4(u0.z, u0.w, inv),
+                                        quant4(u1.x, u1.y, inv), quant4(u1.z, u1.w, inv))
+                           : make_uint4(0u, 0u, 0u, 0u);
+      };
+      int row = row_t, rem = rem_t;
+#pragma unroll
+      for (int j = 0; j < kKeep; ++j) {
+        if (t + 64 * j < chunks && row < n_tok) put(row, rem, quant16(keep[2 * j], keep[2 * j + 1]));
+        rem += 64;
+        while (rem >= per_row) {
+          rem -= per_row;
+          ++row;
+        }
+      }
+      for (int c = t + 64 * kKeep; c < chunks && row < n_tok; c += 64) {
+        const uint4* src = xv + ((static_cast<long long>(row) * a.K + (kb0 + (rem >> 3)) * 128 + (rem & 7) * 16) >> 3);
+        put(row, rem, quant16(__ldcg(src), __ldcg(src + 1)));
         rem += 64;
         while (rem >= per_row) {
           rem -= per_row;
@@ -458,6 +503,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   }
 
   // ---- epilogue: TMEM -> shared partials -> cluster reduction -> bf16 ----------
+  if (a.coop && warp < 2) cluster_wait();  // the split barrier's first phase (the stagers waited already)
   if (!mbar_wait(done, 0, budget, nullptr)) set_status(a.status, kStatusTimeout);
   tc_fence_after();
   pdl_wait();
@@ -497,11 +543,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       const int kk = it - m * rows;
       const int orow = rank * Qr + kk;
       const int tok = routed ? misc->tokens[m] : m;
-      float g = 0.0f;
-      float u = 0.0f;
-      for (int p = 0; p < S; ++p) {
-        g += recv[((p * SUBS + 0) * npad + m) * Qr + kk];
-        if (kSwiglu) u += recv[((p * SUBS + 1) * npad + m) * Qr + kk];
+      // the S partials: every load issued up front (indices past S clamped to
+      // rank 0's slot, in bounds, and not added), then summed in rank order
+      float gp[8], up[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const int pp = p < S ? p : 0;
+        gp[p] = recv[((pp * SUBS + 0) * npad + m) * Qr + kk];
+        up[p] = kSwiglu ? recv[((pp * SUBS + 1) * npad + m) * Qr + kk] : 0.0f;
+      }
+      float g = gp[0];
+      float u = up[0];
+#pragma unroll
+      for (int p = 1; p < 8; ++p) {
+        if (p < S) {
+          g += gp[p];
+          u += up[p];
+        }
       }
       if (kSwiglu) {
         const float yg = g * scale;
@@ -652,7 +710,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   if (recv_bytes > 20 * 1024 || S == 1) recv_bytes = 0;
   const int misc_bytes = static_cast<int>((sizeof(GemmMisc) + 15) & ~static_cast<size_t>(15)) + recv_bytes;
   auto smem_for = [&](int st) {
-    return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 2 + 2 * kBStages) * 8 + misc_bytes;
+    return 1024 + st * kSubBytes + bsm_bytes + (2 * st + 3 + 2 * kBStages) * 8 + misc_bytes;
   };
   // the deepest ring (<= 6 stages) that keeps two CTAs per SM, else 6 stages at one CTA per SM
   int stages = 6;
@@ -686,6 +744,14 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   a.bsm_bytes = bsm_bytes;
   a.tmem_cols = tmem_cols;
   a.recv_bytes = recv_bytes;
+  // The fused quantiser shares the amax across the cluster once all of x no
+  // longer arrives in one batch of loads per thread (16 vectors of 8 values
+  // for each of the 64 stager threads) and each CTA's slice fits its kept
+  // registers (5 chunks of 16 values per thread: M = 4 at K = 5120).
+  a.coop = (g.x != nullptr && S > 1 && static_cast<long long>(g.M) * g.K > 64 * 16 * 8 &&
+            static_cast<long long>(g.M) * nkb_max * 8 <= 64 * 5)
+               ? 1
+               : 0;
   a.debug = g.debug ? 1 : 0;
 
   Launch L(dim3(S, n_tiles, g.slots), dim3(kGemmThreads), static_cast<size_t>(smem), s,
