@@ -213,6 +213,11 @@ __device__ __forceinline__ void dsmem_st_async_f32x2(uint32_t addr, float x, flo
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// Arrive without release semantics: for a phase that only orders mbarrier
+// initialisations, which fence.mbarrier_init.release.cluster has published.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -228,11 +228,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
-  // Cooperative quantiser: first phase of a split cluster barrier.  Every
-  // thread arrives here; the stagers wait before they store into a peer's
-  // shared memory (so every peer's barriers are initialised), the other warps
-  // wait before the epilogue's cluster barrier.
-  if (a.coop) cluster_arrive();
+  // First phase of a split cluster barrier: every thread arrives here, and
+  // waits before it first stores into a peer's shared memory (so every peer's
+  // barriers are initialised; thread 0 published them with
+  // fence.mbarrier_init before the block barrier above, hence a relaxed
+  // arrive): the cooperative quantiser's stagers before they send their slice
+  // maxima, every other thread at the epilogue.
+  if (S > 1) cluster_arrive_relaxed();
 
   if (warp == 0) {
     // ---- weight producer ----
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   }
 
   // ---- epilogue: TMEM -> shared partials -> cluster reduction -> bf16 ----------
-  if (a.coop && warp < 2) cluster_wait();  // the split barrier's first phase (the stagers waited already)
+  if (S > 1 && !(a.coop && warp >= 2)) cluster_wait();  // first phase (the cooperative stagers waited already)
   if (!mbar_wait(done, 0, budget, nullptr)) set_status(a.status, kStatusTimeout);
   tc_fence_after();
   pdl_wait();
@@ -513,6 +515,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     // Push: each thread owns one accumulator row (its TMEM lane) and stores it
     // straight into the receive buffer of the CTA that owns that output row;
     // one cluster barrier later every owner holds all S partials locally.
+    // (Non-blocking st.async stores counted on the owner's mbarrier instead of
+    // the barrier were measured slower at M = 1.)
     const int Qr = (128 + S - 1) / S;
     const int row = warp * 32 + lane;
     const int owner = row / Qr;
