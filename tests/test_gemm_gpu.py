@@ -80,6 +80,27 @@ def test_act_quant_codes_and_scale_bit_exact(M, K):
     assert mism.size == 0, f"{len(mism)} codes differ, first {mism[:5].tolist()}"
 
 
+@pytest.mark.parametrize("M,split", [(2, 2), (2, 3), (3, 4), (4, 4), (5, 5), (4, 8), (6, 8), (1, 4)])
+def test_cooperative_quantiser_codes_bit_exact(M, split):
+    """The fused quantiser at M*K > 8192 with a split-K cluster: each CTA loads
+    only its K slice and the cluster exchanges the slice maxima (uneven slices
+    at 3 and 5 CTAs; M = 1 takes the whole-x path).  The published codes and
+    s_x are bit-exact against the oracle's, and the GEMM output holds the GEMM
+    rule."""
+    K, N2 = 5120, 512
+    g = np.random.default_rng(400 + 10 * M + split)
+    x = dg.bf16_normal(g, (M, K))
+    x[M - 1, K - 5:] = dg.bf16_bits(np.float32([0.0, -0.0, 1e-30, 30.0, -2.0]))  # the maximum in the last slice
+    w, s_w = dg.e4m3_weight(g, N2, K)
+    out, ws = run_fc13(x, w, s_w, split=split)
+    xq_ref, sx_ref = oracle.act_quant(x)
+    assert ws[8:12].view(np.float32)[0] == sx_ref
+    xq = ws[256:256 + M * K].reshape(M, K)
+    mism = np.argwhere(xq != xq_ref)
+    assert mism.size == 0, f"{len(mism)} codes differ, first {mism[:5].tolist()}"
+    helpers.check_gemm(out, oracle.fc13_swiglu(x, w, s_w), f"cooperative quantiser M={M} split={split}")
+
+
 def test_act_quant_all_zero_input():
     x = np.zeros((2, 256), dtype=np.uint16)
     g = np.random.default_rng(5)

@@ -5,7 +5,8 @@ step's kernels run from a CUDA graph, so the host launches one graph per step.
 These tests capture the step exactly as the benchmark does (one graph holding
 the PDL-chained steps of two layer replicas), replay it over rotating inputs
 written into the buffers the graph reads, and check every replay's outputs
-against the oracle on the same inputs:
+against the oracle on the same inputs (100 replays of the decode step at the
+tiny and batch-1 shapes):
 
   - DecodeLayer.step (FC_QKV + scaling -> split-KV attention -> FC13 +
     SwiGLU) at tiny, layer_b1 and verify4; verify4 splits each kv head over
@@ -39,6 +40,9 @@ pytestmark = [pytest.mark.gpu,
 
 REPLICAS = 2
 INPUT_SETS = [0, 1, 0]  # the input set written before each checked replay
+# DecodeLayer.step: checked replays per workload, cycling through three input sets
+# (the oracle runs once per set and replica)
+STEP_REPLAYS = {"tiny": 100, "layer_b1": 100, "verify4": 12}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -121,11 +125,14 @@ def test_decode_step_graph_replay_matches_the_oracle(name):
     steps()
     torch.cuda.synchronize()
     graph = capture(steps)
-    for k, j in enumerate(INPUT_SETS):
-        acts = [activation_set(wl, r, j) for r in range(REPLICAS)]
+    sets = {j: [activation_set(wl, r, j) for r in range(REPLICAS)] for j in range(3)}
+    dev_sets = {j: [(dev_u16(a[0]), dev_u16(a[1])) for a in sets[j]] for j in sets}
+    for k in range(STEP_REPLAYS[name]):
+        j = (0, 1, 0, 2)[k % 4]
+        acts = sets[j]
         for r in range(REPLICAS):
-            xin[r][0].copy_(dev_u16(acts[r][0]))
-            xin[r][1].copy_(dev_u16(acts[r][1]))
+            xin[r][0].copy_(dev_sets[j][r][0])
+            xin[r][1].copy_(dev_sets[j][r][1])
             reps[r]["lay"].attn_out.fill_(-1)
             reps[r]["lay"].ffn_out.fill_(-1)
         graph.replay()
@@ -136,14 +143,14 @@ def test_decode_step_graph_replay_matches_the_oracle(name):
             check_step(wl, rep, j, acts[r][0], acts[r][1], host_u16(rep["lay"].attn_out),
                        host_u16(rep["lay"].ffn_out), host_u16(rep["lay"].qkv), f"{name} replay {k} replica {r}")
     # a burst of back-to-back replays with no host synchronisation in between
+    j_last = (0, 1, 0, 2)[(STEP_REPLAYS[name] - 1) % 4]
     for _ in range(8):
         graph.replay()
     torch.cuda.synchronize()
-    acts = [activation_set(wl, r, INPUT_SETS[-1]) for r in range(REPLICAS)]
     for r, rep in enumerate(reps):
         rep["lay"].read_status()
         assert counters_zero(rep["lay"], wl)
-        check_step(wl, rep, INPUT_SETS[-1], acts[r][0], acts[r][1], host_u16(rep["lay"].attn_out),
+        check_step(wl, rep, j_last, sets[j_last][r][0], sets[j_last][r][1], host_u16(rep["lay"].attn_out),
                    host_u16(rep["lay"].ffn_out), None, f"{name} burst replica {r}")
     del graph
 
