@@ -591,14 +591,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     const int row = warp * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int ncols = SUBS * npad;
-    for (int c0 = 0; c0 < ncols; c0 += 32) {  // up to four 8-column loads in flight per wait
-      uint32_t r[4][8];
+    for (int c0 = 0; c0 < ncols; c0 += 64) {  // up to eight 8-column loads in flight per wait
+      uint32_t r[8][8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 8; ++q)
         if (c0 + 8 * q < ncols) tmem_ld_x8(lane_base + static_cast<uint32_t>(c0 + 8 * q), r[q]);
       tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         const int cq = c0 + 8 * q;  // 8 columns of one sub-accumulator (npad is a multiple of 8)
         const int mq = cq - ((SUBS == 2 && cq >= npad) ? npad : 0);
 #pragma unroll
@@ -611,28 +611,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
   cluster_sync();  // all S partial accumulators are complete and visible
 
   const float scale = misc->sx * scale_w;
-  const int r0 = 128 * rank / S;
-  const int rows = 128 * (rank + 1) / S - r0;
-  const int items = rows * n_tok;
+  // This CTA owns output rows [4*g0, 4*(g0+ng)): groups of 4 consecutive rows,
+  // so every peer read is one 16-byte load (a group's partials of one token
+  // are contiguous in the parked [column][128 rows] layout).
+  const int g0 = 32 * rank / S;
+  const int ng = 32 * (rank + 1) / S - g0;
+  const int items = ng * n_tok;  // (token, row group)
   const uint32_t part_base = smem_u32(part);
   // kPullBatch items per thread per round: all their peer loads are issued
   // before the first sum, so a round costs one DSMEM round trip, not one per item.
-  constexpr int kPullBatch = 4;
+  constexpr int kPullBatch = 2;
   for (int it0 = threadIdx.x; it0 < items; it0 += kGemmThreads * kPullBatch) {
-    float gv[kPullBatch][8], uv[kPullBatch][8];
+    float4 gv[kPullBatch][8], uv[kPullBatch][8];
 #pragma unroll
     for (int q = 0; q < kPullBatch; ++q) {
       const int it = it0 + q * kGemmThreads;
-      const int m = it / rows;
-      const int row = r0 + (it - m * rows);
+      const int m = it / ng;
+      const int row = 4 * (g0 + (it - m * ng));
       const uint32_t off_g = part_base + static_cast<uint32_t>((m * 128 + row) * 4);
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        gv[q][p] = 0.0f;
-        uv[q][p] = 0.0f;
+        gv[q][p] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uv[q][p] = gv[q][p];
         if (it < items && p < S) {
-          gv[q][p] = dsmem_ld_f32(dsmem_addr(off_g, p));
-          if (kSwiglu) uv[q][p] = dsmem_ld_f32(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p));
+          gv[q][p] = dsmem_ld_f32x4(dsmem_addr(off_g, p));
+          if (kSwiglu) uv[q][p] = dsmem_ld_f32x4(dsmem_addr(off_g + static_cast<uint32_t>(npad * 128 * 4), p));
         }
       }
     }
@@ -640,29 +643,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     for (int q = 0; q < kPullBatch; ++q) {
       const int it = it0 + q * kGemmThreads;
       if (it >= items) continue;
-      const int m = it / rows;
-      const int row = r0 + (it - m * rows);
+      const int m = it / ng;
+      const int row = 4 * (g0 + (it - m * ng));
       const int tok = routed ? misc->tokens[m] : m;
-      float g = 0.0f;
-      float u = 0.0f;
+      float g[4] = {0.f, 0.f, 0.f, 0.f};
+      float u[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int p = 0; p < 8; ++p) {  // peers summed in rank order
-        g += gv[q][p];
-        u += uv[q][p];
+        g[0] += gv[q][p].x;
+        g[1] += gv[q][p].y;
+        g[2] += gv[q][p].z;
+        g[3] += gv[q][p].w;
+        u[0] += uv[q][p].x;
+        u[1] += uv[q][p].y;
+        u[2] += uv[q][p].z;
+        u[3] += uv[q][p].w;
       }
-      if (kSwiglu) {
-        const float yg = g * scale;
-        const float yu = u * scale;
-        const float o = yg / (1.0f + expf(-yg)) * yu;
-        const __nv_bfloat16 b = __float2bfloat16_rn(o);
-        a.out[static_cast<long long>(tok) * a.ldo + tile * 128 + row] = *reinterpret_cast<const uint16_t*>(&b);
-      } else {
-        const int col = tile * 128 + row;
-        float y = g * scale;
-        if (col < a.q_cols) y *= a.q_scale;
-        const __nv_bfloat16 b = __float2bfloat16_rn(y);
-        a.out[static_cast<long long>(tok) * a.ldo + col] = *reinterpret_cast<const uint16_t*>(&b);
+      float o[4];
+      const int col = tile * 128 + row;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (kSwiglu) {
+          const float yg = g[i] * scale;
+          const float yu = u[i] * scale;
+          o[i] = yg / (1.0f + expf(-yg)) * yu;
+        } else {
+          o[i] = g[i] * scale;
+          if (col + i < a.q_cols) o[i] *= a.q_scale;
+        }
       }
+      uint2 packed;
+      packed.x = pack_bf16x2(o[0], o[1]);
+      packed.y = pack_bf16x2(o[2], o[3]);
+      *reinterpret_cast<uint2*>(a.out + static_cast<long long>(tok) * a.ldo + col) = packed;
     }
   }
   tc_fence_before();
