@@ -156,6 +156,12 @@ def test_graph_replayer_captures_each_length_once_and_replays_in_order():
     assert rp.lengths(20) == [6, 2]
     rp.run(20)
     assert sorted(captures) == [2, 6]  # nothing captured again
+    del log[:]
+    rp.warm(20)  # the untimed replay ahead of a timed run: the plan's first graph, once
+    assert log == list(range(6))
+    del log[:]
+    rp.warm(2)
+    assert log == [0, 1]
 
 
 def test_recorded_traffic_matches_the_current_source_only(tmp_path, monkeypatch):
