@@ -734,6 +734,20 @@ static bool encode_kv_map(CUtensorMap* m, const void* base, int d, int Lcap, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_u8_rows_sw128(CUtensorMap* m, const void* base, int row_bytes, int rows, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr || row_bytes < 128 || row_bytes % 16 != 0 || rows < 1 || box_rows < 1 || box_rows > 256)
+    return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
+                           static_cast<cuuint64_t>(row_bytes) * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Workspace of dl_decode_attn with P clusters per (b, kv head) of S CTAs: the
 // 256-byte header, the per-(head, owner) counters, the per-owner (m, l) of each
 // cluster, and the merged item states of each cluster.

@@ -66,6 +66,12 @@ cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s
 cudaError_t launch_pack(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
                         cudaStream_t s);
 
+// A 2-D TMA map over rows of row_bytes bytes (row pitch row_bytes): boxes of
+// 128 bytes x box_rows rows with the 128-byte swizzle (the tcgen05 SW128
+// K-major operand layout); rows past `rows` read as zeros.  false when the
+// driver's encoder is unavailable or refuses the shape.
+bool encode_u8_rows_sw128(CUtensorMap* m, const void* base, int row_bytes, int rows, int box_rows);
+
 struct GemmLaunch {
   const uint8_t* w;
   long long w_expert_bytes;

@@ -44,6 +44,7 @@ constexpr int kMaxExperts = 1024;
 constexpr int kBStages = 4;       // B ring depth when the activations stream in with the weights
 
 struct GemmArgs {
+  CUtensorMap xq_map;         // tma_b: x_q [M][K] as 128-byte x npad boxes, 128-byte swizzle
   const uint8_t* w;           // packed weights (expert 0 block for MoE)
   long long w_expert_bytes;   // bytes per expert block (0 for dense)
   const float* w_scale;       // [1] or [E]
@@ -61,6 +62,7 @@ struct GemmArgs {
   int tmem_cols;
   int recv_bytes;             // > 0: split-K partials are pushed into a dedicated receive buffer
   int coop;                   // fused quantiser: the cluster shares the amax (each CTA reads its K slice)
+  int tma_b;                  // streamed B (dense): one tensor load per k-block, issued by the producer
   int debug;
 };
 
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
     mbar_init(xready, 64);
     mbar_init(done, 1);
     for (int s = 0; s < kBStages; ++s) {
-      mbar_init(bfull0 + 8u * s, 64);
+      mbar_init(bfull0 + 8u * s, a.tma_b ? 1 : 64);
       mbar_init(bempty0 + 8u * s, 1);
     }
     mbar_init(amaxbar, 1);
@@ -242,11 +244,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       const uint64_t pol = l2_policy_evict_first();
       const int n_issue = a.debug ? nsub - 1 : nsub;  // test hook: withhold the last stage
       int issued = 0;
+      // Streamed B by tensor loads (dense): the activations of k-block kb land
+      // in B slot kb % kBStages with one copy of npad rows x 128 bytes (the
+      // tensor map swizzles them into the operand layout and zero-fills the
+      // padding rows).  They exist only once the preceding kernel has written
+      // them, so the first `stages` weight blocks are issued before the PDL
+      // wait and their k-blocks' activations right after it; from then on each
+      // k-block's activations go out just ahead of its first weight block.
+      const bool tma_b = a.tma_b != 0;
+      const int prefill = a.stages < n_issue ? a.stages : n_issue;
+      int kb_b = 0;  // next k-block whose activations are to be issued
+      auto issue_b = [&](int kb) -> bool {
+        const int bs = kb % kBStages;
+        if (kb >= kBStages &&
+            !mbar_wait(bempty0 + 8u * bs, static_cast<uint32_t>((kb / kBStages) - 1) & 1u, budget, abort_flag))
+          return false;
+        mbar_arrive_expect_tx(bfull0 + 8u * bs, static_cast<uint32_t>(npad * 128));
+        tma_load_3d(smem_u32(bsm + bs * npad * 128), &a.xq_map, (kb0 + kb) * 128, 0, 0, bfull0 + 8u * bs);
+        return true;
+      };
+      auto issue_b_upto = [&](int kb_end) -> bool {  // k-blocks kb_b .. kb_end - 1
+        for (; kb_b < kb_end; ++kb_b)
+          if (!issue_b(kb_b)) return false;
+        return true;
+      };
+      if (tma_b) prefetch_tensormap(&a.xq_map);
       // stage s and round parity kept incrementally (no division by the
       // runtime ring depth on this single-thread issue path)
       int s = 0;
       uint32_t round_par = 0;  // (i / stages) & 1
       for (int i = 0; i < n_issue; ++i) {
+        if (tma_b && i >= prefill) {
+          if (i == prefill) pdl_wait();  // x_q is written by the preceding kernel
+          if (!issue_b_upto(i / SUBS + 1)) {
+            set_status(a.status, kStatusTimeout);
+            *abort_flag = 1;
+            break;
+          }
+        }
         if (i >= a.stages && !mbar_wait(empty0 + 8u * s, round_par ^ 1u, budget, abort_flag)) {
           set_status(a.status, kStatusTimeout);
           *abort_flag = 1;
@@ -261,10 +296,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
           round_par ^= 1u;
         }
       }
+      if (tma_b && !*abort_flag) {  // the activations of every k-block not issued yet
+        if (prefill >= n_issue) pdl_wait();
+        if (!issue_b_upto(nkb)) {
+          set_status(a.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+      }
       if (*abort_flag) {  // let the copies still in flight land before the CTA can exit
         const int first = issued > a.stages ? issued - a.stages : 0;
         for (int i = first; i < issued; ++i)
           mbar_wait(full0 + 8u * (i % a.stages), static_cast<uint32_t>(i / a.stages) & 1u, budget, nullptr);
+        for (int kb = kb_b > kBStages ? kb_b - kBStages : 0; kb < kb_b; ++kb)
+          mbar_wait(bfull0 + 8u * (kb % kBStages), static_cast<uint32_t>(kb / kBStages) & 1u, budget, nullptr);
       }
     }
     __syncwarp();
@@ -455,6 +499,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       mbar_arrive(xready);
     } else {
     if (t == 0) misc->sx = __ldcg(a.s_x);
+    if (!a.tma_b) {
     // Stream the e4m3 activations of each k-block into the B ring with 16-byte
     // async copies, one commit group per k-block, kBStages-1 k-blocks in
     // flight: a block is published (bfull) as soon as its own group has landed,
@@ -501,6 +546,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_e4m3_kernel(const __grid
       ++committed;
     }
     cp_async_wait_pending(0);  // nothing in flight when the stager moves on
+    }
     }
   }
 
@@ -740,7 +786,7 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
   // TMEM safety: the CTAs that can share an SM must fit in its 512 columns.
   while ((233472 / (smem + 1024)) * tmem_cols > 512) smem += 1024;
 
-  GemmArgs a;
+  GemmArgs a{};
   a.w = g.w;
   a.w_expert_bytes = g.w_expert_bytes;
   a.w_scale = g.w_scale;
@@ -770,6 +816,12 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t s) {
                ? 1
                : 0;
   a.debug = g.debug ? 1 : 0;
+  // Dense streamed activations come in by tensor loads (routed tokens are
+  // gathered row by row by the stager warps instead)
+  a.tma_b = (stream_b && g.expert_ids == nullptr &&
+             encode_u8_rows_sw128(&a.xq_map, g.xq, g.K, g.M, npad_max))
+                ? 1
+                : 0;
 
   Launch L(dim3(S, n_tiles, g.slots), dim3(kGemmThreads), static_cast<size_t>(smem), s,
            static_cast<unsigned>(S), g.pdl);

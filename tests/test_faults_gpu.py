@@ -39,8 +39,10 @@ def _fc13_case(seed=1, M=2, K=512, N2=256):
     return x, w, s_w, wp
 
 
-def test_gemm_timeout_is_reported_and_context_stays_usable():
-    x, w, s_w, wp = _fc13_case()
+@pytest.mark.parametrize("M,K", [(2, 512), (64, 1024)])
+def test_gemm_timeout_is_reported_and_context_stays_usable(M, K):
+    # (64, 1024): x_q is streamed into the GEMM by tensor loads beside the weights
+    x, w, s_w, wp = _fc13_case(M=M, K=K)
     M, K = x.shape
     N2 = w.shape[0]
     out = torch.empty((M, N2 // 2), dtype=torch.int16, device="cuda")
@@ -54,9 +56,14 @@ def test_gemm_timeout_is_reported_and_context_stays_usable():
     helpers.check_gemm(host_u16(out), oracle.fc13_swiglu(x, w, s_w), "after timeout")
 
 
-def test_qkv_timeout_with_a_single_stage_per_cta():
+@pytest.mark.parametrize("M", [1, 64])
+def test_qkv_timeout_with_a_single_stage_per_cta(M):
+    # N = 256, one k-block per CTA: no weight block is loaded at all (at M = 64,
+    # K = 1024, M*K is past the fused quantiser and the k-block's activations
+    # still arrive by their tensor load)
     g = np.random.default_rng(3)
-    M, K, Hq, Hkv, d = 1, 512, 2, 1, 64  # N = 256, one k-block per CTA: nothing is loaded at all
+    K, Hq, Hkv, d = (512 if M == 1 else 1024), 2, 1, 64
+    split = K // 128 if M > 1 else 4
     N = (Hq + 2 * Hkv) * d
     x = dg.bf16_normal(g, (M, K))
     w, s_w = dg.e4m3_weight(g, N, K)
@@ -65,7 +72,7 @@ def test_qkv_timeout_with_a_single_stage_per_cta():
     dl.check(dl.dl_pack_fp8_weight(wd, wp, N, K, dl.DL_PACK_PLAIN))
     out = torch.empty((M, N), dtype=torch.int16, device="cuda")
     ws, n = new_ws(M, K)
-    flags = dl.DL_FLAG_DEBUG_TIMEOUT | (4 << dl.DL_FLAG_SPLIT_SHIFT)
+    flags = dl.DL_FLAG_DEBUG_TIMEOUT | (split << dl.DL_FLAG_SPLIT_SHIFT)
     assert dl.dl_fc_qkv_scale(dev_u16(x), M, K, wp, dev_f32(s_w), Hq, Hkv, d, 0.125, out, ws, n,
                               flags=flags) == dl.DL_OK
     assert dl.dl_read_status(ws) == dl.DL_ERR_TIMEOUT

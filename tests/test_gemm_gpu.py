@@ -139,6 +139,20 @@ def test_fc13_split_k_cluster_sizes(split):
     helpers.check_gemm(out, oracle.fc13_swiglu(x, w, s_w), f"fc13 split={split}")
 
 
+@pytest.mark.parametrize("M,split", [(7, 0), (13, 3), (40, 5), (64, 1), (64, 8)])
+def test_fc13_streamed_activations_by_tensor_loads(M, split):
+    # M*K > 32768: x is quantised by its own kernel and each k-block of x_q
+    # reaches the GEMM by one tensor load (padding rows M..npad-1 zero-filled
+    # by the copy), over uneven split-K slices and a B ring that wraps 10 times
+    # at split 1
+    g = np.random.default_rng(600 + M + split)
+    K, N2 = 5120, 512
+    x = dg.bf16_normal(g, (M, K))
+    w, s_w = dg.e4m3_weight(g, N2, K)
+    out, _ = run_fc13(x, w, s_w, split=split)
+    helpers.check_gemm(out, oracle.fc13_swiglu(x, w, s_w), f"fc13 streamed B M={M} split={split}")
+
+
 def test_fc13_pdl_flag_does_not_change_bits():
     g = np.random.default_rng(7)
     x = dg.bf16_normal(g, (4, 512))
