@@ -71,13 +71,6 @@ struct AttnArgs {
   int debug;
 };
 
-// Two e4m3 codes (low byte first) -> f16x2 (low half first); exact, since every
-// e4m3 value is an f16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-}
-
 // 4 bytes at (row, col) of a V^T tile of KT-byte rows as TMA lays it out: the
 // 128-byte swizzle for 128-byte rows, the 64-byte swizzle for 64-byte rows
 // (16-byte chunk index XOR row bits; col is a multiple of 4).
@@ -86,6 +79,16 @@ __device__ __forceinline__ uint32_t vt_word(const uint8_t* vt, int row, int col)
   static_assert(KT == 64 || KT == 128, "V^T rows of 64 or 128 bytes");
   const int ch = KT == 128 ? (((col >> 4) ^ row) & 7) : (((col >> 4) ^ (row >> 1)) & 3);
   return *reinterpret_cast<const uint32_t*>(vt + row * KT + (ch << 4) + (col & 15));
+}
+
+// The four e4m3 codes of a 32-bit word (low byte first) -> two f16x2 words
+// (codes 0-1, then 2-3; low half first).  Exact, since every e4m3 value is an
+// f16 value.  The word's halves are the 16-bit operands of the two
+// conversions directly: masking or shifting them out first cost two more
+// instructions per pair on the attention's critical path.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t ld_b32(const uint16_t* p) {
@@ -346,8 +349,9 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
           for (int ks = 0; ks < KS; ++ks) {
             const uint32_t wA = (&kA[ks >> 2].x)[ks & 3];
             const uint32_t wB = (&kB[ks >> 2].x)[ks & 3];
-            const uint32_t a0 = e4m3x2_to_f16x2(wA & 0xFFFFu), a2 = e4m3x2_to_f16x2(wA >> 16);
-            const uint32_t a1 = e4m3x2_to_f16x2(wB & 0xFFFFu), a3 = e4m3x2_to_f16x2(wB >> 16);
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_f16x2x2(wA, a0, a2);
+            e4m3x4_to_f16x2x2(wB, a1, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const uint2 qf = qs[(ks * NT + nt) * 32 + lane];
@@ -374,35 +378,57 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         // ---- online softmax (log2 domain) ----
         const int kA = key_base + pA;  // physical keys of MMA rows g and g+8
         const int kB = key_base + pB;
+        // A tile that every row sees in full (any but a chunk's last and the
+        // causal diagonal) needs no mask: padding rows then see it too, but
+        // their states are never stored.
+        const bool full = key_base + 16 <= hi && key_base + 15 <= L - a.T;
+        float x[NT][4];
+        bool raise = false;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            x[nt][j] = (full || (kA < hi && kA <= lim[nt][j])) ? sc[nt][j] * scale_log2 : -INFINITY;
+            x[nt][2 + j] = (full || (kB < hi && kB <= lim[nt][j])) ? sc[nt][2 + j] * scale_log2 : -INFINITY;
+            const float thr = m_run[nt][j] + static_cast<float>(kLazyRescale);
+            raise = raise || x[nt][j] > thr || x[nt][2 + j] > thr;
+          }
+        // Lazy rescale: the reference max m_run of a row moves only when this
+        // tile's row max exceeds it by more than 2^kLazyRescale, so the O
+        // rescale below is rarely needed and p stays <= 2^kLazyRescale, far
+        // from overflow.  Whether any score of the warp exceeds its row's
+        // threshold is one vote; only then are the row maxima taken (three
+        // shuffle rounds per row) and the rows that need it rescaled.
+        if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              float mx = fmaxf(x[nt][j], x[nt][2 + j]);
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              if (mx > m_run[nt][j] + static_cast<float>(kLazyRescale)) {
+                const float alpha = ex2(m_run[nt][j] - mx);  // 0 when m_run is -inf
+                l_run[nt][j] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                  o[mt][nt][j] *= alpha;
+                  o[mt][nt][2 + j] *= alpha;
+                }
+                m_run[nt][j] = mx;
+              }
+            }
+        }
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           float p[4];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const float x0 = (kA < hi && kA <= lim[nt][j]) ? sc[nt][j] * scale_log2 : -INFINITY;
-            const float x1 = (kB < hi && kB <= lim[nt][j]) ? sc[nt][2 + j] * scale_log2 : -INFINITY;
-            float mx = fmaxf(x0, x1);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            // Lazy rescale: the reference max m_run moves only when this tile's
-            // max exceeds it by more than 2^kLazyRescale, so the O rescale below
-            // is rarely needed; p stays <= 2^kLazyRescale, far from overflow.
-            if (mx > m_run[nt][j] + static_cast<float>(kLazyRescale)) {
-              const float m_new = mx;
-              const float alpha = ex2(m_run[nt][j] - m_new);  // 0 when m_run is -inf
-              l_run[nt][j] *= alpha;
-#pragma unroll
-              for (int mt = 0; mt < KS; ++mt) {
-                o[mt][nt][j] *= alpha;
-                o[mt][nt][2 + j] *= alpha;
-              }
-              m_run[nt][j] = m_new;
-            }
             const float m_use = (m_run[nt][j] == -INFINITY) ? 0.0f : m_run[nt][j];
-            p[j] = ex2(x0 - m_use);
-            p[2 + j] = ex2(x1 - m_use);
+            p[j] = ex2(x[nt][j] - m_use);
+            p[2 + j] = ex2(x[nt][2 + j] - m_use);
             l_run[nt][j] += p[j] + p[2 + j];
           }
           // P^T as the B operand [k = key][n = row]: transpose each 8x8 block
@@ -420,8 +446,9 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
             const int r0 = 16 * mt + g, r1 = r0 + 8;
             const uint32_t w0 = vt_word<kAttnKT>(vt, r0, col);
             const uint32_t w1 = vt_word<kAttnKT>(vt, r1, col);
-            const uint32_t a0 = e4m3x2_to_f16x2(w0 & 0xFFFFu), a2 = e4m3x2_to_f16x2(w0 >> 16);
-            const uint32_t a1 = e4m3x2_to_f16x2(w1 & 0xFFFFu), a3 = e4m3x2_to_f16x2(w1 >> 16);
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_f16x2x2(w0, a0, a2);
+            e4m3x4_to_f16x2x2(w1, a1, a3);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
           }
