@@ -71,16 +71,6 @@ struct AttnArgs {
   int debug;
 };
 
-// 4 bytes at (row, col) of a V^T tile of KT-byte rows as TMA lays it out: the
-// 128-byte swizzle for 128-byte rows, the 64-byte swizzle for 64-byte rows
-// (16-byte chunk index XOR row bits; col is a multiple of 4).
-template <int KT>
-__device__ __forceinline__ uint32_t vt_word(const uint8_t* vt, int row, int col) {
-  static_assert(KT == 64 || KT == 128, "V^T rows of 64 or 128 bytes");
-  const int ch = KT == 128 ? (((col >> 4) ^ row) & 7) : (((col >> 4) ^ (row >> 1)) & 3);
-  return *reinterpret_cast<const uint32_t*>(vt + row * KT + (ch << 4) + (col & 15));
-}
-
 // The four e4m3 codes of a 32-bit word (low byte first) -> two f16x2 words
 // (codes 0-1, then 2-3; low half first).  Exact, since every e4m3 value is an
 // f16 value.  The word's halves are the 16-bit operands of the two
@@ -439,18 +429,29 @@ __global__ void __launch_bounds__(32 * (W + 1), W == 4 ? 2 : 1)
         if (F8) {
           // V^T rows 16mt+g and 16mt+g+8 (d), bytes warp*16 + 4t .. +3 = MMA keys
           // 2t, 2t+1 (e = 0, 1) and 2t+8, 2t+9 (e = 2, 3)
-          const uint8_t* vt = ring + s * STAGE_BYTES + KV_BYTES;
-          const int col = warp * 16 + 4 * q4;
+          // Two m-tiles per ldmatrix: lane l addresses row l % 8 of matrix l / 8,
+          // matrices 0-3 being V^T rows 16mt + {0, 8} and 16(mt+1) + {0, 8}.  A
+          // matrix row is this warp's 16-byte chunk (keys warp*16 .. +15) of a
+          // V^T row as TMA swizzled it: chunk index XOR the row's low 3 bits
+          // (128-byte rows) or bits 1-2 (64-byte rows).  Thread t of group g so
+          // receives bytes 4t .. 4t+3 of that chunk in row g of each matrix.
+          const int mi = lane >> 3, rr = lane & 7;
+          const int vch = kAttnKT == 128 ? ((warp ^ rr) & 7) : ((warp ^ (rr >> 1)) & 3);
+          const uint32_t vaddr = smem_u32(ring + s * STAGE_BYTES + KV_BYTES) +
+                                 static_cast<uint32_t>((16 * (mi >> 1) + 8 * (mi & 1) + rr) * kAttnKT + (vch << 4));
 #pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            const int r0 = 16 * mt + g, r1 = r0 + 8;
-            const uint32_t w0 = vt_word<kAttnKT>(vt, r0, col);
-            const uint32_t w1 = vt_word<kAttnKT>(vt, r1, col);
-            uint32_t a0, a1, a2, a3;
-            e4m3x4_to_f16x2x2(w0, a0, a2);
-            e4m3x4_to_f16x2x2(w1, a1, a3);
+          for (int mt = 0; mt < KS; mt += 2) {
+            uint32_t w[4];
+            ldsm_x4(vaddr + static_cast<uint32_t>(mt * 16 * kAttnKT), w[0], w[1], w[2], w[3]);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            for (int h = 0; h < 2; ++h) {
+              uint32_t a0, a1, a2, a3;
+              e4m3x4_to_f16x2x2(w[2 * h], a0, a2);
+              e4m3x4_to_f16x2x2(w[2 * h + 1], a1, a3);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                mma_f16_16816(o[mt + h][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
           }
         } else {
           const int j = lane >> 3;
