@@ -53,11 +53,6 @@ __global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __g
   __shared__ float red[kNqWarps];
   __shared__ float cta_amax;
 
-  // x and r may be produced by the preceding kernel: wait before reading them,
-  // then let the dependent GEMM start streaming its weights.
-  pdl_wait();
-  pdl_trigger();
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int C = gridDim.x;
@@ -74,6 +69,20 @@ __global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __g
   const uint4* rv = a.r != nullptr ? reinterpret_cast<const uint4*>(a.r) + rbase : nullptr;
   uint4* hv = a.h_out != nullptr ? reinterpret_cast<uint4*>(a.h_out) + rbase : nullptr;
   const uint4* gv = reinterpret_cast<const uint4*>(a.gamma);
+
+  // gamma is a static input: its vectors are loaded before the wait for the
+  // preceding kernel, so they are in registers when the norm needs them
+  uint4 gk[kNqKeep];
+#pragma unroll
+  for (int j = 0; j < kNqKeep; ++j) {
+    const int v = tr + j * TPR;
+    gk[j] = (live && v < VR) ? __ldg(gv + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  // x and r may be produced by the preceding kernel: wait before reading them,
+  // then let the dependent GEMM start streaming its weights.
+  pdl_wait();
+  pdl_trigger();
 
   // ---- h = x (+ r), kept in registers; row sum of squares -------------------
   uint4 h[kNqKeep];
@@ -116,7 +125,7 @@ __global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __g
 #pragma unroll
   for (int j = 0; j < kNqKeep; ++j) {
     const int v = tr + j * TPR;
-    if (live && v < VR) m = fmaxf(m, norm8(h[j], __ldg(gv + v), rs, y));
+    if (live && v < VR) m = fmaxf(m, norm8(h[j], gk[j], rs, y));
   }
   for (int v = tr + kNqKeep * TPR; live && v < VR; v += TPR) {
     const uint4 u = reload_h(xv, rv, hv, v);
@@ -144,7 +153,7 @@ __global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __g
   for (int j = 0; j < kNqKeep; ++j) {
     const int v = tr + j * TPR;
     if (live && v < VR) {
-      norm8(h[j], __ldg(gv + v), rs, y);
+      norm8(h[j], gk[j], rs, y);
       q2[v] = amax > 0.0f ? quant8(y, inv) : make_uint2(0u, 0u);
     }
   }
@@ -160,11 +169,17 @@ __global__ void __launch_bounds__(kNqThreads) add_rmsnorm_quant_kernel(const __g
 
 cudaError_t launch_add_rmsnorm_quant(const uint16_t* x, const uint16_t* r, uint16_t* h_out, const uint16_t* gamma,
                                      int M, int K, float eps, uint8_t* xq, float* s_x, cudaStream_t s, bool pdl) {
-  // rows per CTA: the smallest power of two that fits M rows in <= 8 CTAs
+  // rows per CTA: the smallest power of two that fits M rows in <= 16 CTAs
+  // (a cluster above 8 CTAs is non-portable; more CTAs shorten each one's
+  // share of the loads at large M)
   int R = 1;
-  while (R < 16 && (M + R - 1) / R > 8) R <<= 1;
+  while (R < 16 && (M + R - 1) / R > 16) R <<= 1;
   const int C = (M + R - 1) / R;
-  if (C > 8) return cudaErrorInvalidValue;
+  if (C > 16) return cudaErrorInvalidValue;
+  if (C > 8) {
+    cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(add_rmsnorm_quant_kernel), 0, true);
+    if (e != cudaSuccess) return e;
+  }
   NormQuantArgs a;
   a.x = x;
   a.r = r;
