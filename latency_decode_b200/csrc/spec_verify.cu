@@ -40,31 +40,29 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// -0 and +0 are the same logit value: -0 is keyed as +0, so that a tie between
-// them, like any other tie, goes to the lower index.
-__device__ __forceinline__ unsigned long long sv_key(uint32_t bf16_bits, int index) {
-  if (bf16_bits == 0x8000u) bf16_bits = 0u;
-  return (static_cast<unsigned long long>(ordered_bits(__uint_as_float(bf16_bits << 16))) << 32) |
+// (logit, index) as one key: order-preserving value bits above, the inverted
+// index below, so that the larger key is the larger logit and, among equal
+// logits, the lower index.  -0 and +0 are the same logit value: -0 is keyed as
+// +0, so that a tie between them, like any other tie, goes to the lower index.
+__device__ __forceinline__ unsigned long long sv_key(float v, int index) {
+  if (v == 0.0f) v = 0.0f;
+  return (static_cast<unsigned long long>(ordered_bits(v)) << 32) |
          static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(index));
 }
 
-// Best key among the 8 bf16 logits of one 16-byte vector starting at index v8.
-__device__ __forceinline__ unsigned long long best8(uint4 u, int v8) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  unsigned long long k = 0ull;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const unsigned long long lo = sv_key(w[i] & 0xFFFFu, v8 + 2 * i);
-    const unsigned long long hi = sv_key(w[i] >> 16, v8 + 2 * i + 1);
-    k = lo > k ? lo : k;
-    k = hi > k ? hi : k;
-  }
-  return k;
+__device__ __forceinline__ float bf16_at(uint4 u, int e) {  // element e (0..7) of 8 packed bf16
+  const uint32_t w = e < 2 ? u.x : e < 4 ? u.y : e < 6 ? u.z : u.w;
+  return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
-// Launched as grid (C, B) with clusters of (C, 1, 1).
-__global__ void __launch_bounds__(kSvThreads) spec_verify_kernel(const __grid_constant__ VerifyArgs a) {
+// Launched as grid (C, B) with clusters of (C, 1, 1).  kMinBlocks = 2 caps the
+// registers at 64 so that two CTAs share an SM (a 16-CTA cluster then spans 8
+// SMs of a GPC and grids beyond one CTA per SM run in one wave); grids that
+// fit one CTA per SM use the unconstrained build, which is faster there.
+template <int kMinBlocks>
+__global__ void __launch_bounds__(kSvThreads, kMinBlocks) spec_verify_kernel(const __grid_constant__ VerifyArgs a) {
   __shared__ unsigned long long best[kSvMaxT];
+  __shared__ unsigned long long wbest[kSvThreads / 32];
 
   // the logits are the output of the preceding kernel (the LM head)
   pdl_wait();
@@ -78,39 +76,69 @@ __global__ void __launch_bounds__(kSvThreads) spec_verify_kernel(const __grid_co
   const int c0 = static_cast<int>(static_cast<long long>(nv) * r / C);
   const int c1 = static_cast<int>(static_cast<long long>(nv) * (r + 1) / C);
   const int per = c1 - c0;  // vectors of this CTA's slice, per row
-  if (threadIdx.x < T) best[threadIdx.x] = 0ull;
-  __syncthreads();
-
   const uint4* base = reinterpret_cast<const uint4*>(a.logits) + static_cast<long long>(b) * T * nv;
-  const int items = per * T;  // (row, vector) pairs, row-major
-  int cur_row = -1;
-  unsigned long long cur = 0ull;
-  for (int i0 = threadIdx.x; i0 < items; i0 += kSvThreads * kSvBatch) {
-    uint4 u[kSvBatch];
+  // Each of the T rows gets its own group of G = 512 / T' threads (T' = T
+  // rounded up to a power of two; groups past T idle), which scans the row's
+  // slice with 16-byte loads, kSvBatch in flight per thread.  A thread meets
+  // its vectors in increasing index order, so only a strictly larger value
+  // replaces its best one (the first of equal values stays); the row's best
+  // over the group is then the largest (value, lowest index) key, reduced by
+  // shuffles and, for groups wider than a warp, one shared slot per warp.
+  int Tp = 1;
+  while (Tp < T) Tp <<= 1;
+  const int G = kSvThreads / Tp;
+  const int t = threadIdx.x / G;
+  const int gi = threadIdx.x - t * G;
+  float best_v = 0.0f;
+  int best_i = -1;
+  if (t < T) {
+    const uint4* row = base + static_cast<long long>(t) * nv + c0;
+    for (int v0 = gi; v0 < per; v0 += G * kSvBatch) {
+      uint4 u[kSvBatch];
 #pragma unroll
-    for (int j = 0; j < kSvBatch; ++j) {
-      const int i = i0 + j * kSvThreads;
-      if (i < items) {
-        const int t = i / per;
-        u[j] = __ldcg(base + static_cast<long long>(t) * nv + c0 + (i - t * per));
-      }
-    }
+      for (int j = 0; j < kSvBatch; ++j)
+        if (v0 + j * G < per) u[j] = __ldcg(row + v0 + j * G);
 #pragma unroll
-    for (int j = 0; j < kSvBatch; ++j) {
-      const int i = i0 + j * kSvThreads;
-      if (i < items) {
-        const int t = i / per;
-        if (t != cur_row) {
-          if (cur_row >= 0) atomicMax(&best[cur_row], cur);
-          cur_row = t;
-          cur = 0ull;
+      for (int j = 0; j < kSvBatch; ++j) {
+        if (v0 + j * G < per) {
+          // the vector's largest value (packed bf16 maxima), then, only when it
+          // beats the best so far, its first position
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+          const __nv_bfloat162 m2 = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+          const float vmax = fmaxf(__low2float(m2), __high2float(m2));
+          if (best_i < 0 || vmax > best_v) {
+            int e = 7;
+#pragma unroll
+            for (int k = 6; k >= 0; --k)
+              if (bf16_at(u[j], k) == vmax) e = k;
+            best_v = vmax;
+            best_i = (c0 + v0 + j * G) * 8 + e;
+          }
         }
-        const unsigned long long k = best8(u[j], (c0 + (i - t * per)) * 8);
-        cur = k > cur ? k : cur;
       }
     }
   }
-  if (cur_row >= 0) atomicMax(&best[cur_row], cur);
+  unsigned long long key = best_i >= 0 ? sv_key(best_v, best_i) : 0ull;
+  const int width = G < 32 ? G : 32;  // G is a power of two >= 16
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    if (o < width) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+      key = other > key ? other : key;
+    }
+  }
+  const int warp = threadIdx.x >> 5;
+  if (G <= 32) {
+    if (t < T && gi == 0) best[t] = key;
+  } else {
+    if ((threadIdx.x & 31) == 0) wbest[warp] = key;
+  }
+  __syncthreads();
+  if (G > 32 && threadIdx.x < T) {  // the G / 32 warps of row threadIdx.x
+    unsigned long long k = 0ull;
+    for (int w = threadIdx.x * (G / 32); w < (threadIdx.x + 1) * (G / 32); ++w) k = wbest[w] > k ? wbest[w] : k;
+    best[threadIdx.x] = k;
+  }
   cluster_sync();  // every CTA's row maxima are final and visible cluster-wide
 
   if (r == 0 && threadIdx.x < 32) {
@@ -151,8 +179,11 @@ cudaError_t launch_spec_verify(const uint16_t* logits, int B, int T, int V, cons
   if (C < 1) C = 1;
   const int nv = V / 8;
   if (C > nv) C = nv;
+  const bool two = static_cast<long long>(C) * B > sm_count();
+  const void* fn = two ? reinterpret_cast<const void*>(spec_verify_kernel<2>)
+                       : reinterpret_cast<const void*>(spec_verify_kernel<1>);
   if (C > 8) {
-    cudaError_t e = ensure_kernel_attrs(reinterpret_cast<const void*>(spec_verify_kernel), 0, true);
+    cudaError_t e = ensure_kernel_attrs(fn, 0, true);
     if (e != cudaSuccess) return e;
   }
   VerifyArgs a;
@@ -166,7 +197,7 @@ cudaError_t launch_spec_verify(const uint16_t* logits, int B, int T, int V, cons
   a.T = T;
   a.V = V;
   Launch L(dim3(C, B), dim3(kSvThreads), 0, s, static_cast<unsigned>(C), pdl);
-  return cudaLaunchKernelEx(&L.cfg, spec_verify_kernel, a);
+  return two ? cudaLaunchKernelEx(&L.cfg, spec_verify_kernel<2>, a) : cudaLaunchKernelEx(&L.cfg, spec_verify_kernel<1>, a);
 }
 
 }  // namespace dl
