@@ -101,7 +101,7 @@ def test_signed_zero_tie_lowest_index_wins(golden_dir):
 
 
 @pytest.mark.parametrize("B,T,V", [(1, 4, 1000), (3, 4, 4096), (16, 4, 32000), (64, 2, 2048), (5, 8, 800),
-                                   (2, 32, 128), (1, 1, 64)])
+                                   (2, 32, 128), (1, 1, 64), (3, 3, 5000), (2, 5, 70000), (1, 17, 3000)])
 def test_every_accept_length(B, T, V):
     g = np.random.default_rng(B * 100 + T * 7 + V)
     lg, draft = planted(g, B, T, V, list(range(T)))
@@ -122,6 +122,25 @@ def test_ties_lowest_index_wins_across_cta_slices():
     draft = np.array([[5, 101024, 9], [0, 0, 0]], dtype=np.int32)
     nacc = check(lg, draft, None, "ties")
     assert nacc.tolist() == [2, 3]
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_ties_between_threads_and_warps_of_one_row_slice(T):
+    # equal maxima in vectors that different threads and different warps of
+    # one CTA's row group scan (8 logits per vector; the group has 512 / T
+    # threads), and equal maxima at +0 / -0: the lowest index wins in each row
+    g = np.random.default_rng(11 + T)
+    B, V = 1, 202048
+    lg = dg.bf16_normal(g, (B, T, V))
+    big = dg.bf16_bits(np.float32([50.0]))[0]
+    expect = []
+    for t in range(T):
+        idx = [8 * (7 + 40 * t) + 3, 8 * (1 + 40 * t) + 6, 8 * (300 + 40 * t) + 1]  # vectors 1, 7, 300 (+40 t)
+        lg[0, t, idx] = big
+        expect.append(min(idx))
+    draft = np.array([expect[:T - 1]], dtype=np.int32)
+    nacc = check(lg, draft, None, f"ties across threads T={T}")
+    assert nacc.tolist() == [T - 1]
 
 
 @pytest.mark.parametrize("name", ["verify4", "batch16x4"])
