@@ -154,9 +154,6 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
   else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
   else asm volatile("cp.async.wait_group 3;" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
 
 // ---- cluster / distributed shared memory ----------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
