@@ -79,6 +79,10 @@ typedef enum dl_status {
                                      s_x, written into this same workspace by
                                      dl_add_rmsnorm_quant; the GEMM skips its activation
                                      quantisation and `x` may be NULL */
+#define DL_FLAG_COPY_NO_WAIT 16u   /* dl_copy only: the copy neither reads what the kernel
+                                     before it in the stream writes nor writes what that
+                                     kernel reads, so under DL_FLAG_PDL it starts without
+                                     waiting for it (the caller vouches for this) */
 #define DL_FLAG_SPLIT_SHIFT 8     /* bits [8,13): if non-zero, force the GEMM split-K
                                      cluster size (1..8), or the number of clusters per
                                      (b, kv head) of dl_decode_attn (1..16), instead of
@@ -388,8 +392,11 @@ size_t dl_decode_attn_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int 
  *             aligned, not overlapping
  *   bytes     a multiple of 16 (0 launches nothing)
  * With DL_FLAG_PDL the kernel waits for its predecessor before it reads src or
- * writes dst.  Host memory written this way is visible to the host once the
- * stream has been synchronised.
+ * writes dst, unless DL_FLAG_COPY_NO_WAIT says that neither is touched by that
+ * predecessor: then it runs beside it (an upload beside the previous step's
+ * download uses both directions of the host link at once).  Host memory
+ * written this way is visible to the host once the stream has been
+ * synchronised.
  * ------------------------------------------------------------------------- */
 dl_status dl_copy(const void* src, void* dst, size_t bytes, void* stream, unsigned flags);
 

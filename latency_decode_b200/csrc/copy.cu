@@ -18,9 +18,10 @@ constexpr int kCopyThreads = 256;
 constexpr int kCopyBatch = 4;  // 16-byte loads in flight per thread per round
 
 __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                          long long n16) {
-  // src may be written, and dst still read, by the preceding kernel
-  pdl_wait();
+                                                          long long n16, int wait_first) {
+  // src may be written, and dst still read, by the preceding kernel, unless
+  // the caller has vouched that neither is
+  if (wait_first) pdl_wait();
   pdl_trigger();
   const long long stride = static_cast<long long>(gridDim.x) * kCopyThreads;
   for (long long i0 = blockIdx.x * static_cast<long long>(kCopyThreads) + threadIdx.x; i0 < n16;
@@ -39,14 +40,14 @@ __global__ void __launch_bounds__(kCopyThreads) copy_kernel(const uint4* __restr
   }
 }
 
-cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s, bool pdl) {
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s, bool pdl, bool wait_first) {
   const long long n16 = static_cast<long long>(bytes / 16);
   if (n16 == 0) return cudaSuccess;
   long long blocks = (n16 + kCopyThreads * kCopyBatch - 1) / (kCopyThreads * kCopyBatch);
   if (blocks > 2ll * sm_count()) blocks = 2ll * sm_count();
   Launch L(dim3(static_cast<unsigned>(blocks)), dim3(kCopyThreads), 0, s, 0, pdl);
   return cudaLaunchKernelEx(&L.cfg, copy_kernel, reinterpret_cast<const uint4*>(src), reinterpret_cast<uint4*>(dst),
-                            n16);
+                            n16, wait_first ? 1 : 0);
 }
 
 }  // namespace dl

@@ -453,7 +453,8 @@ dl_status dl_copy(const void* src, void* dst, size_t bytes, void* stream, unsign
   if (!aligned(src, 16) || !aligned(dst, 16) || bytes % 16 != 0) return DL_ERR_ALIGNMENT;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(src), b0 = reinterpret_cast<uintptr_t>(dst);
   if (bytes > 0 && a0 < b0 + bytes && b0 < a0 + bytes) return DL_ERR_INVALID_ARG;  // overlap
-  return cuda_status(dl::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream), (flags & DL_FLAG_PDL) != 0));
+  return cuda_status(dl::launch_copy(src, dst, bytes, static_cast<cudaStream_t>(stream), (flags & DL_FLAG_PDL) != 0,
+                                     (flags & DL_FLAG_COPY_NO_WAIT) == 0));
 }
 
 dl_status dl_read_status(void* ws, void* stream) {

@@ -62,7 +62,7 @@ cudaError_t launch_add_rmsnorm_quant(const uint16_t* x, const uint16_t* r, uint1
 cudaError_t launch_spec_verify(const uint16_t* logits, int B, int T, int V, const int32_t* draft,
                                int32_t* target_ids, int32_t* n_accepted, int32_t* emitted, int32_t* seq_lens,
                                cudaStream_t s, bool pdl);
-cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s, bool pdl);
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s, bool pdl, bool wait_first);
 cudaError_t launch_pack(const uint8_t* w_nk, uint8_t* w_packed, int N, int K, int kind,
                         cudaStream_t s);
 

@@ -29,6 +29,7 @@ DL_ERR_DEVICE_ARG = 7
 DL_FLAG_PDL = 1
 DL_FLAG_DEBUG_TIMEOUT = 2
 DL_FLAG_XQ_READY = 4
+DL_FLAG_COPY_NO_WAIT = 16
 DL_FLAG_SPLIT_SHIFT = 8
 DL_PACK_PLAIN = 0
 DL_PACK_SWIGLU = 1

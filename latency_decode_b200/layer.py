@@ -78,15 +78,23 @@ class DecodeLayer:
                                    stream=stream, flags=flags))
 
     def step_host(self, x_host: torch.Tensor, out_host: torch.Tensor, k_cache, v_cache, seq_lens, stream=None,
-                  flags: int = dl.DL_FLAG_PDL) -> None:
+                  flags: int = dl.DL_FLAG_PDL, overlap_upload: bool = False) -> None:
         """One step whose activations come from, and whose results go to, pinned
         host memory: x_host is [2, M, K] bf16 bits (x1, x2) from cudaHostAlloc
         (torch's pin_memory), out_host has the layout of self.out_buf.  The two
         transfers are kernels of the same PDL chain (dl_copy), so the QKV GEMM
-        streams its weights while the activations arrive."""
+        streams its weights while the activations arrive.
+
+        overlap_upload: the kernel just before this call in the stream is the
+        result download of a previous step_host (of this or another
+        DecodeLayer), which reads only that layer's out_buf and writes its host
+        buffer; the upload then starts beside it (DL_FLAG_COPY_NO_WAIT), using
+        the other direction of the host link.  That download waited for its
+        step's kernels before it let this one start, so x_dev is free."""
         if not hasattr(self, "x_dev"):
             self.x_dev = torch.empty((2, self.M, self.K), dtype=torch.int16, device=self.device)
-        dl.check(dl.dl_copy(x_host, self.x_dev, self.x_dev.numel() * 2, stream=stream, flags=flags))
+        up_flags = flags | (dl.DL_FLAG_COPY_NO_WAIT if overlap_upload else 0)
+        dl.check(dl.dl_copy(x_host, self.x_dev, self.x_dev.numel() * 2, stream=stream, flags=up_flags))
         self.step(self.x_dev[0], self.x_dev[1], k_cache, v_cache, seq_lens, stream=stream, flags=flags)
         dl.check(dl.dl_copy(self.out_buf, out_host, self.out_buf.numel() * 2, stream=stream, flags=flags))
 

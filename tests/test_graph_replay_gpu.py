@@ -155,10 +155,12 @@ def test_decode_step_graph_replay_matches_the_oracle(name):
     del graph
 
 
-@pytest.mark.parametrize("name", ["tiny", "layer_b1"])
-def test_step_host_graph_replay_matches_the_oracle(name):
+@pytest.mark.parametrize("name,overlap", [("tiny", False), ("layer_b1", False), ("tiny", True), ("layer_b1", True)])
+def test_step_host_graph_replay_matches_the_oracle(name, overlap):
     """Activations from pinned host memory, results to pinned host memory, the
-    transfers being copy kernels of the same PDL chain inside the graph."""
+    transfers being copy kernels of the same PDL chain inside the graph (with
+    overlap, each replica's upload runs beside the previous replica's
+    download, DL_FLAG_COPY_NO_WAIT)."""
     wl = dg.WORKLOADS[name]
     reps = build_layers(wl)
     hx = [torch.empty((2, wl.M, wl.K), dtype=torch.int16).pin_memory() for _ in range(REPLICAS)]
@@ -167,7 +169,7 @@ def test_step_host_graph_replay_matches_the_oracle(name):
     def steps():
         for r, rep in enumerate(reps):
             rep["lay"].step_host(hx[r], hout[r], rep["k"], rep["v"], rep["sl"],
-                                 stream=torch.cuda.current_stream().cuda_stream)
+                                 stream=torch.cuda.current_stream().cuda_stream, overlap_upload=overlap)
 
     def write_inputs(j):
         acts = [activation_set(wl, r, j) for r in range(REPLICAS)]
