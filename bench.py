@@ -998,6 +998,17 @@ def run_ours(args):
         e2e_graph_step(i)
     us_e2e, e2e_kind, e2e_lengths = per_call_us(e2e_graph_step, G, args.steps)
     us_e2e = max_over_ranks(us_e2e)
+
+    # The same with every upload waiting for the previous step's download, as a
+    # decode loop whose next input depends on the last result has to run
+    def e2e_graph_step_seq(i):
+        r = i % R
+        layers[r].step_host(hx, hout, kvs[r][0], kvs[r][1], seq_lens,
+                            stream=torch.cuda.current_stream().cuda_stream)
+
+    for i in range(3):
+        e2e_graph_step_seq(i)
+    us_e2e_seq = max_over_ranks(per_call_us(e2e_graph_step_seq, G, args.steps)[0])
     if e2e_kind == "graph":
         e2e_mode = (f"CUDA graphs of {' and '.join(map(str, e2e_lengths))} steps, each: copy kernel host->device "
                     "(beside the previous step's download), the chain, copy kernel device->host")
@@ -1062,7 +1073,9 @@ def run_ours(args):
         "layer_alg_bytes": wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes,
         "layer_achieved_gbs": (wl.n_qkv * wl.K + wl.N2 * wl.K + kv_bytes) / (us_layer * 1e-6) / 1e9,
         "e2e": {"value": us_e2e, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "mode": e2e_mode, "direct_launch_us": us_e2e_direct},
+                "mode": e2e_mode, "direct_launch_us": us_e2e_direct,
+                "sequential_us": us_e2e_seq,
+                "sequential_mode": "as value, but each upload waits for the previous step's download"},
         "cpu_baseline": cpu,
         "cpu_baseline_all_cores": cpu_all,
         "gpu_launches": (2 * gl + 1) * args.steps,
