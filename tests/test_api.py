@@ -29,6 +29,17 @@ def declared_entry_points():
     return sorted(set(re.findall(r"^\s*(?:dl_status|size_t|const char\*)\s+(dl_\w+)\s*\(", text, re.M)))
 
 
+def test_binding_constants_match_the_header():
+    """Every DL_* integer macro of include/dl.h (flags, pack kinds, status codes)
+    has the same value in the Python binding."""
+    text = open(os.path.join(ROOT, "include", "dl.h")).read()
+    macros = dict((name, int(val)) for name, val in re.findall(r"^#define\s+(DL_\w+)\s+(\d+)u?\b", text, re.M))
+    macros.update((name, int(val)) for name, val in re.findall(r"^\s*(DL_(?:OK|ERR_\w+))\s*=\s*(\d+)", text, re.M))
+    assert "DL_FLAG_PDL" in macros and "DL_FLAG_COPY_NO_WAIT" in macros and "DL_ERR_DEVICE_ARG" in macros
+    for name, val in macros.items():
+        assert getattr(dl, name) == val, name
+
+
 def test_exports_every_declared_entry_point():
     names = declared_entry_points()
     assert len(names) >= 8
